@@ -1,0 +1,691 @@
+"""Benchmark of the fine-grained online FP8 hot path on B200.
+
+One step = one pass of the hot path over one batch of synthetic input.
+Workloads (``--workload``):
+  ffn    (default) dense FFN up-projection forward: X bf16 [4096x7168] and
+         W bf16 [7168x18432] quantized online (1x128 / 128x128, scales
+         computed on every step), block-scaled FP8 GEMM -> bf16 [4096x18432].
+         3 launches per step.  value = 2MNK / step time (TFLOP/s).
+  quant  quantize-only bandwidth: act [8192x7168] and weight [7168x18432]
+         bf16.  value = bytes moved / step time (GB/s).
+  moe    MoE expert GEMMs, 8192 tokens x top-8 of 256 experts: act quant of
+         the routed tokens, grouped gate+up GEMM (N=4096, K=7168), act quant
+         of the down input, grouped down GEMM (N=7168, K=2048).  Expert
+         weights are quantized once before timing.  value in TFLOP/s.
+  dgrad  backward dgrad: dY bf16 [16384x18432] quantized 1x128 along N, W
+         [7168x18432] quantized (untransposed), dX = dY W^T -> bf16.
+
+Contract: ``python bench.py --gpus N --steps K --warmup W`` (N > 1 under
+torchrun, one rank per GPU) prints one JSON line on rank 0.  Each rank runs
+its own replica of the workload (data parallel over tokens: no collective on
+the data path); the time is the max over ranks of the CUDA-event time of K
+steps, taken between barriers and device synchronizations.
+``--impl reference`` times the plain CPU oracle instead, on a bounded
+sample of the same workload (rank 0 only).
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "FP8 block-scaled GEMM TFLOP/s & quantize GB/s, % of B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_OVER_BF16 = 2.0     # nominal dense ratio, 4.5 / 2.25 PFLOP/s
+CSRC = os.path.join(ROOT, "fp8_fine_grained_online_b200", "csrc")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC)):
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    cur = kernel_source_hash()
+    with open(TRAFFIC_FILE) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and not line.startswith("#"):
+                k, w, b, src_hash = parts[:4]
+                if k == kernel and w == workload and src_hash == cur:
+                    return float(b)
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.idx = device_index
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(device_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- workloads
+
+class Workload:
+    name = ""
+    unit = "TFLOP/s"
+    dominant = ""
+
+    def launches_per_step(self):
+        return len(self.kernels)
+
+    def work_per_step(self):
+        """Units of `value` per step (FLOP or bytes)."""
+        raise NotImplementedError
+
+
+class FFN(Workload):
+    """Online-quantized dense FFN up-projection forward."""
+    name = synth.FFN.name
+    unit = "TFLOP/s"
+    dominant = "blockscaled_gemm"
+
+    def __init__(self, fp8, device, M=4096, K=7168, N=18432):
+        self.fp8, self.M, self.K, self.N = fp8, M, K, N
+        self.kernels = ["quant_act_1x128", "quant_weight_128x128", "blockscaled_gemm"]
+        if device is None:
+            return
+        self.x, self.w = synth.ffn_inputs(device, M, K, N)
+        self.qx = torch.empty((M, K), dtype=torch.uint8, device=device)
+        self.sx = torch.empty((M, K // 128), dtype=torch.float32, device=device)
+        self.qw = torch.empty((N, K), dtype=torch.uint8, device=device)
+        self.sw = torch.empty((K // 128, N // 128), dtype=torch.float32, device=device)
+        self.c = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+
+    def config(self):
+        return {"workload": self.name, "M": self.M, "N": self.N, "K": self.K,
+                "x": "bf16 [%dx%d] N(0,1) 0.1%% outliers x100" % (self.M, self.K),
+                "w": "bf16 [%dx%d] N(0,0.02)" % (self.K, self.N), "out": "bf16",
+                "l2": "inputs larger than L2 (X+W bf16 = %.0f MB > 126 MB)" %
+                      ((self.M * self.K + self.K * self.N) * 2 / 1e6)}
+
+    def flops(self):
+        return 2.0 * self.M * self.N * self.K
+
+    def work_per_step(self):
+        return self.flops()
+
+    def algorithmic(self):
+        """Per launch: (kind, amount) -- bytes for HBM-bound kernels, FLOPs for the GEMM."""
+        M, N, K = self.M, self.N, self.K
+        return {
+            "quant_act_1x128": ("bytes", M * K * 2 + M * K + M * (K // 128) * 4),
+            "quant_weight_128x128": ("bytes", K * N * 2 + K * N + (K // 128) * (N // 128) * 4),
+            "blockscaled_gemm": ("flops", 2.0 * M * N * K),
+        }
+
+    def step(self, marks):
+        f = self.fp8
+        marks(0)
+        f.fp8_quantize_act_1x128(self.x, q=self.qx, sa=self.sx)
+        marks(1)
+        f.fp8_quantize_weight_128x128(self.w, transpose_out=True, q=self.qw, sb=self.sw)
+        marks(2)
+        f.fp8_blockscaled_gemm(self.qx, self.sx, self.qw, self.sw, c=self.c)
+        marks(3)
+
+    # end to end through the public API with pinned host buffers
+    def e2e_setup(self):
+        self.hx = self.x.cpu().pin_memory()
+        self.hw = self.w.cpu().pin_memory()
+        self.hc = torch.empty((self.M, self.N), dtype=torch.bfloat16, pin_memory=True)
+        return self.hx.numel() * 2 + self.hw.numel() * 2, self.hc.numel() * 2
+
+    def e2e_step(self):
+        self.fp8.e2e_linear_forward(self.hx, self.hw, out_host=self.hc)
+
+    def oracle_sample(self, orc, rows, nbs):
+        """Oracle on a sample of the step: quantize `rows` rows of X and the
+        `nbs` 128-column blocks of W, GEMM those rows x columns.  Returns the
+        FLOPs of the sampled GEMM (the unit the step is counted in)."""
+        xs = synth.ffn_inputs("cpu", M=self.M, K=self.K, N=self.N) if not hasattr(self, "_cpu") \
+            else self._cpu
+        self._cpu = xs
+        x, w = xs
+        xa = x[:rows].contiguous().view(torch.int16).numpy().view(np.uint16)
+        qa, sa = orc.quantize_act_1x128(xa)
+        flops = 0.0
+        for nb in range(nbs):
+            blk = w[:, nb * 128:(nb + 1) * 128].contiguous().view(torch.int16).numpy().view(np.uint16)
+            qb, sb = orc.quantize_weight_128x128(blk, transpose_out=True)
+            orc.gemm_ref(qa, sa, qb, sb)
+            flops += 2.0 * rows * 128 * self.K
+        return flops
+
+
+class Quant(Workload):
+    name = synth.QUANT.name
+    unit = "GB/s"
+    dominant = "quant_weight_128x128"
+
+    def __init__(self, fp8, device, M=8192, K=7168, N=18432):
+        self.fp8, self.M, self.K, self.N = fp8, M, K, N
+        self.kernels = ["quant_act_1x128", "quant_weight_128x128"]
+        if device is None:
+            return
+        self.x, self.w = synth.quant_inputs(device)
+        self.qx = torch.empty((M, K), dtype=torch.uint8, device=device)
+        self.sx = torch.empty((M, K // 128), dtype=torch.float32, device=device)
+        self.qw = torch.empty((N, K), dtype=torch.uint8, device=device)
+        self.sw = torch.empty((K // 128, N // 128), dtype=torch.float32, device=device)
+
+    def config(self):
+        return {"workload": self.name, "act": "bf16 [%dx%d]" % (self.M, self.K),
+                "weight": "bf16 [%dx%d] -> E4M3 [N,K]" % (self.K, self.N),
+                "dist": "N(0,0.02), 0.1% outliers x100",
+                "l2": "weight input 264 MB > L2; the weight pass evicts the act input"}
+
+    def algorithmic(self):
+        M, N, K = self.M, self.N, self.K
+        return {
+            "quant_act_1x128": ("bytes", M * K * 2 + M * K + M * (K // 128) * 4),
+            "quant_weight_128x128": ("bytes", K * N * 2 + K * N + (K // 128) * (N // 128) * 4),
+        }
+
+    def work_per_step(self):
+        return sum(v for _, v in self.algorithmic().values())
+
+    def step(self, marks):
+        f = self.fp8
+        marks(0)
+        f.fp8_quantize_act_1x128(self.x, q=self.qx, sa=self.sx)
+        marks(1)
+        f.fp8_quantize_weight_128x128(self.w, transpose_out=True, q=self.qw, sb=self.sw)
+        marks(2)
+
+    def e2e_setup(self):
+        self.hx = self.x.cpu().pin_memory()
+        self.hw = self.w.cpu().pin_memory()
+        self.hqx = torch.empty_like(self.qx, device="cpu").pin_memory()
+        self.hqw = torch.empty_like(self.qw, device="cpu").pin_memory()
+        self.hsx = torch.empty_like(self.sx, device="cpu").pin_memory()
+        self.hsw = torch.empty_like(self.sw, device="cpu").pin_memory()
+        return ((self.hx.numel() + self.hw.numel()) * 2,
+                self.hqx.numel() + self.hqw.numel() + (self.hsx.numel() + self.hsw.numel()) * 4)
+
+    def e2e_step(self):
+        f = self.fp8
+        x = self.hx.to("cuda", non_blocking=True)
+        w = self.hw.to("cuda", non_blocking=True)
+        qx, sx = f.fp8_quantize_act_1x128(x)
+        qw, sw = f.fp8_quantize_weight_128x128(w, transpose_out=True)
+        for h, d in ((self.hqx, qx), (self.hsx, sx), (self.hqw, qw), (self.hsw, sw)):
+            h.copy_(d, non_blocking=True)
+
+    def oracle_sample(self, orc, rows, nbs):
+        x, w = synth.quant_inputs("cpu") if not hasattr(self, "_cpu") else self._cpu
+        self._cpu = (x, w)
+        xa = x[:rows * 8].contiguous().view(torch.int16).numpy().view(np.uint16)
+        orc.quantize_act_1x128(xa)
+        moved = xa.size * 3 + xa.shape[0] * (xa.shape[1] // 128) * 4
+        blk = w[:, :nbs * 128].contiguous().view(torch.int16).numpy().view(np.uint16)
+        orc.quantize_weight_128x128(blk, transpose_out=True)
+        moved += blk.size * 3 + (blk.shape[0] // 128) * (blk.shape[1] // 128) * 4
+        return float(moved)
+
+
+class DGrad(FFN):
+    """dX = dY W^T with W quantized untransposed (K-major for this product)."""
+    name = synth.DGRAD.name
+
+    def __init__(self, fp8, device, M=16384, K=18432, N=7168):
+        self.fp8, self.M, self.K, self.N = fp8, M, K, N
+        self.kernels = ["quant_act_1x128", "quant_weight_128x128", "blockscaled_gemm"]
+        if device is None:
+            return
+        self.x, self.w = synth.dgrad_inputs(device, M, K, N)    # dY [M,K], W [N,K]
+        self.qx = torch.empty((M, K), dtype=torch.uint8, device=device)
+        self.sx = torch.empty((M, K // 128), dtype=torch.float32, device=device)
+        self.qw = torch.empty((N, K), dtype=torch.uint8, device=device)
+        self.sw = torch.empty((N // 128, K // 128), dtype=torch.float32, device=device)
+        self.c = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+
+    def config(self):
+        return {"workload": self.name, "M": self.M, "N": self.N, "K": self.K,
+                "dY": "bf16 [%dx%d] N(0,1e-3) 0.1%% outliers x100" % (self.M, self.K),
+                "W": "bf16 [%dx%d] N(0,0.02), 128x128 blocks read transposed" % (self.N, self.K),
+                "out": "bf16", "l2": "inputs larger than L2 (dY 604 MB)"}
+
+    def algorithmic(self):
+        M, N, K = self.M, self.N, self.K
+        return {
+            "quant_act_1x128": ("bytes", M * K * 2 + M * K + M * (K // 128) * 4),
+            "quant_weight_128x128": ("bytes", K * N * 2 + K * N + (K // 128) * (N // 128) * 4),
+            "blockscaled_gemm": ("flops", 2.0 * M * N * K),
+        }
+
+    def step(self, marks):
+        f = self.fp8
+        marks(0)
+        f.fp8_quantize_act_1x128(self.x, q=self.qx, sa=self.sx)
+        marks(1)
+        f.fp8_quantize_weight_128x128(self.w, transpose_out=False, q=self.qw, sb=self.sw)
+        marks(2)
+        f.fp8_blockscaled_gemm(self.qx, self.sx, self.qw, self.sw, c=self.c, sb_kb_nb=False)
+        marks(3)
+
+    def e2e_setup(self):
+        self.hx = self.x.cpu().pin_memory()
+        self.hw = self.w.cpu().pin_memory()
+        self.hc = torch.empty((self.M, self.N), dtype=torch.bfloat16, pin_memory=True)
+        return (self.hx.numel() + self.hw.numel()) * 2, self.hc.numel() * 2
+
+    def e2e_step(self):
+        f = self.fp8
+        x = self.hx.to("cuda", non_blocking=True)
+        w = self.hw.to("cuda", non_blocking=True)
+        qx, sx = f.fp8_quantize_act_1x128(x)
+        qw, sw = f.fp8_quantize_weight_128x128(w, transpose_out=False)
+        c = f.fp8_blockscaled_gemm(qx, sx, qw, sw, sb_kb_nb=False)
+        self.hc.copy_(c, non_blocking=True)
+
+    def oracle_sample(self, orc, rows, nbs):
+        dy, w = synth.dgrad_inputs("cpu", self.M, self.K, self.N) if not hasattr(self, "_cpu") \
+            else self._cpu
+        self._cpu = (dy, w)
+        xa = dy[:rows].contiguous().view(torch.int16).numpy().view(np.uint16)
+        qa, sa = orc.quantize_act_1x128(xa)
+        flops = 0.0
+        for nb in range(nbs):
+            blk = w[nb * 128:(nb + 1) * 128].contiguous().view(torch.int16).numpy().view(np.uint16)
+            qb, sb = orc.quantize_weight_128x128(blk, transpose_out=False)
+            orc.gemm_ref(qa, sa, qb, sb, b_kmajor=True, sb_transposed=True)
+            flops += 2.0 * rows * 128 * self.K
+        return flops
+
+
+class MoE(Workload):
+    name = synth.MOE.name
+    unit = "TFLOP/s"
+    dominant = "grouped_gemm_gate_up"
+
+    def __init__(self, fp8, device, tokens=8192, experts=256, topk=8, hidden=7168, inter=2048):
+        self.fp8 = fp8
+        self.T, self.E, self.k, self.H, self.I = tokens, experts, topk, hidden, inter
+        self.R = tokens * topk
+        self.kernels = ["quant_act_1x128_x", "grouped_gemm_gate_up", "quant_act_1x128_h",
+                        "grouped_gemm_down"]
+        if device is None:
+            return
+        d = synth.moe_inputs(device, tokens, experts, topk, hidden, inter, with_weights=False)
+        self.x, self.h, self.off = d["x_routed"], d["h_down"], d["offsets"]
+        R, H, I, E = self.R, hidden, inter, experts
+        self.qgu = torch.empty((E, 2 * I, H), dtype=torch.uint8, device=device)
+        self.sgu = torch.empty((E, H // 128, 2 * I // 128), dtype=torch.float32, device=device)
+        self.qdn = torch.empty((E, H, I), dtype=torch.uint8, device=device)
+        self.sdn = torch.empty((E, I // 128, H // 128), dtype=torch.float32, device=device)
+        for e in range(E):   # expert weights: quantized once, outside the timed region
+            w = synth.moe_expert_weight(e, "gate_up", device, hidden, inter)
+            fp8.fp8_quantize_weight_128x128(w, transpose_out=True, q=self.qgu[e], sb=self.sgu[e])
+            w = synth.moe_expert_weight(e, "down", device, hidden, inter)
+            fp8.fp8_quantize_weight_128x128(w, transpose_out=True, q=self.qdn[e], sb=self.sdn[e])
+        del w
+        self.qx = torch.empty((R, H), dtype=torch.uint8, device=device)
+        self.sx = torch.empty((R, H // 128), dtype=torch.float32, device=device)
+        self.qh = torch.empty((R, I), dtype=torch.uint8, device=device)
+        self.sh = torch.empty((R, I // 128), dtype=torch.float32, device=device)
+        self.cgu = torch.empty((R, 2 * I), dtype=torch.bfloat16, device=device)
+        self.cdn = torch.empty((R, H), dtype=torch.bfloat16, device=device)
+        torch.cuda.synchronize()
+
+    def config(self):
+        return {"workload": self.name, "tokens": self.T, "experts": self.E, "topk": self.k,
+                "routed_rows": self.R, "gate_up": "K=%d N=%d" % (self.H, 2 * self.I),
+                "down": "K=%d N=%d" % (self.I, self.H), "out": "bf16",
+                "weights": "quantized once before timing (11.27 GB E4M3)",
+                "l2": "expert weights 11.27 GB >> L2"}
+
+    def algorithmic(self):
+        R, H, I, E = self.R, self.H, self.I, self.E
+        return {
+            "quant_act_1x128_x": ("bytes", R * H * 3 + R * (H // 128) * 4),
+            "grouped_gemm_gate_up": ("flops", 2.0 * R * 2 * I * H),
+            "quant_act_1x128_h": ("bytes", R * I * 3 + R * (I // 128) * 4),
+            "grouped_gemm_down": ("flops", 2.0 * R * H * I),
+        }
+
+    def hbm_bytes(self, kernel):
+        R, H, I, E = self.R, self.H, self.I, self.E
+        if kernel == "grouped_gemm_gate_up":
+            return E * 2 * I * H + R * H + R * 2 * I * 2
+        if kernel == "grouped_gemm_down":
+            return E * H * I + R * I + R * H * 2
+        return None
+
+    def work_per_step(self):
+        return 2.0 * self.R * 2 * self.I * self.H + 2.0 * self.R * self.H * self.I
+
+    def step(self, marks):
+        f = self.fp8
+        marks(0)
+        f.fp8_quantize_act_1x128(self.x, q=self.qx, sa=self.sx)
+        marks(1)
+        f.fp8_grouped_gemm(self.qx, self.sx, self.qgu, self.sgu, self.off, c=self.cgu)
+        marks(2)
+        f.fp8_quantize_act_1x128(self.h, q=self.qh, sa=self.sh)
+        marks(3)
+        f.fp8_grouped_gemm(self.qh, self.sh, self.qdn, self.sdn, self.off, c=self.cdn)
+        marks(4)
+
+    def e2e_setup(self):
+        self.hx = self.x.cpu().pin_memory()
+        self.hh = self.h.cpu().pin_memory()
+        self.hoff = self.off.cpu().pin_memory()
+        self.hgu = torch.empty_like(self.cgu, device="cpu").pin_memory()
+        self.hdn = torch.empty_like(self.cdn, device="cpu").pin_memory()
+        return ((self.hx.numel() + self.hh.numel()) * 2 + self.hoff.numel() * 4,
+                (self.hgu.numel() + self.hdn.numel()) * 2)
+
+    def e2e_step(self):
+        f = self.fp8
+        x = self.hx.to("cuda", non_blocking=True)
+        h = self.hh.to("cuda", non_blocking=True)
+        off = self.hoff.to("cuda", non_blocking=True)
+        qx, sx = f.fp8_quantize_act_1x128(x)
+        cgu = f.fp8_grouped_gemm(qx, sx, self.qgu, self.sgu, off)
+        qh, sh = f.fp8_quantize_act_1x128(h)
+        cdn = f.fp8_grouped_gemm(qh, sh, self.qdn, self.sdn, off)
+        self.hgu.copy_(cgu, non_blocking=True)
+        self.hdn.copy_(cdn, non_blocking=True)
+
+    def oracle_sample(self, orc, rows, nbs):
+        """Expert 0's first `rows` routed rows x `nbs` column blocks of both GEMMs."""
+        if not hasattr(self, "_cpu"):
+            d = synth.moe_inputs("cpu", self.T, self.E, self.k, self.H, self.I, with_weights=False)
+            self._cpu = (d, synth.moe_expert_weight(0, "gate_up", "cpu", self.H, self.I),
+                         synth.moe_expert_weight(0, "down", "cpu", self.H, self.I))
+        d, wgu, wdn = self._cpu
+        flops = 0.0
+        for a, w, K in ((d["x_routed"], wgu, self.H), (d["h_down"], wdn, self.I)):
+            xa = a[:rows].contiguous().view(torch.int16).numpy().view(np.uint16)
+            qa, sa = orc.quantize_act_1x128(xa)
+            for nb in range(nbs):
+                blk = w[:, nb * 128:(nb + 1) * 128].contiguous().view(torch.int16).numpy() \
+                    .view(np.uint16)
+                qb, sb = orc.quantize_weight_128x128(blk, transpose_out=True)
+                orc.gemm_ref(qa, sa, qb, sb)
+                flops += 2.0 * rows * 128 * K
+        return flops
+
+
+WORKLOADS = {"ffn": FFN, "quant": Quant, "moe": MoE, "dgrad": DGrad}
+# Oracle sample per step: (rows, column blocks), sized for a few seconds per step.
+ORACLE_SAMPLE = {"ffn": (32, 2), "quant": (16, 4), "moe": (32, 1), "dgrad": (16, 1)}
+# The single CPU-baseline measurement of the default run: ~10 s of oracle work.
+CPU_BASELINE_SAMPLE = {"ffn": (128, 12), "quant": (64, 24), "moe": (128, 6), "dgrad": (64, 4)}
+
+
+# ----------------------------------------------------------------------------- timing
+
+def run_ours(args, rank, world, local_rank):
+    import fp8_fine_grained_online_b200 as fp8
+    device = "cuda:%d" % local_rank
+    torch.cuda.set_device(local_rank)
+    wl = WORKLOADS[args.workload](fp8, device)
+    stream = torch.cuda.current_stream()
+    nk = len(wl.kernels)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        wl.step(lambda i: None)
+    torch.cuda.synchronize()
+    if fp8.fp8_get_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(torch.cuda.current_device())
+    time.sleep(0.3)
+    wall0 = time.perf_counter()
+    start.record(stream)
+    for s in range(args.steps):
+        wl.step(lambda i, s=s: ev[s][i].record(stream))
+    stop.record(stream)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    barrier()
+    clk = clocks.stop()
+    elapsed_ms = start.elapsed_time(stop)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    dev_err = fp8.fp8_get_device_error()
+
+    per_kernel = {}
+    for i, k in enumerate(wl.kernels):
+        per_kernel[k] = statistics.fmean(ev[s][i].elapsed_time(ev[s][i + 1])
+                                         for s in range(args.steps))
+
+    # end to end through the public API, pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        h2d, d2h = wl.e2e_setup()
+        wl.e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(1, min(args.steps, 5))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(n_e2e):
+            wl.e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=device)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": round(world * wl.work_per_step() * n_e2e / (e_ms / 1e3) / scale(wl), 3),
+               "unit": wl.unit, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": n_e2e}
+    return wl, elapsed_ms, per_kernel, clk, e2e, wall, dev_err
+
+
+def scale(wl):
+    return 1e12 if wl.unit == "TFLOP/s" else 1e9
+
+
+def roofline_entry(wl, kernel, ms, peaks, peak_src):
+    kind, amount = wl.algorithmic()[kernel]
+    if kind == "flops" and wl.unit == "TFLOP/s" and hasattr(wl, "hbm_bytes") \
+            and wl.hbm_bytes(kernel) is not None:
+        # grouped GEMM: weight streaming; report the bound that limits it
+        t_flop = amount / (peaks["bf16_tflops"] * FP8_OVER_BF16 * 1e12)
+        t_hbm = wl.hbm_bytes(kernel) / (peaks["hbm_gbs"] * 1e9)
+        if t_hbm > t_flop:
+            ach = wl.hbm_bytes(kernel) / (ms / 1e3) / 1e9
+            return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
+                    "basis": "HBM bytes of fp8 weights + act + out per launch, %s copy peak" %
+                             peak_src}
+    if kind == "flops":
+        peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+        ach = amount / (ms / 1e3) / 1e12
+        return {"bound": "tensor", "achieved": round(ach, 1), "peak": round(peak, 1),
+                "unit": "TFLOP/s", "frac": round(ach / peak, 4),
+                "basis": "%s bf16 burst x 2 (fp8/bf16 nominal dense ratio)" % peak_src}
+    ach = amount / (ms / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(ach / peaks["hbm_gbs"], 4), "basis": "%s copy peak" % peak_src}
+
+
+def cpu_baseline(args, wl_cls):
+    import oracle
+    wl = wl_cls(None, None)
+    rows, nbs = CPU_BASELINE_SAMPLE[args.workload]
+    wl.oracle_sample(oracle, 1, 1)              # input generation + library load, untimed
+    t0 = time.perf_counter()
+    work = wl.oracle_sample(oracle, rows, nbs)
+    dt = time.perf_counter() - t0
+    return {"value": round(work / dt / scale(wl), 6), "unit": wl.unit,
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "%d rows x %d 128-column blocks of the step, with their online "
+                      "quantization (%.1f s)" % (rows, nbs, dt)}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="ffn")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    wl_cls = WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        import oracle
+        wl = wl_cls(None, None)
+        rows, nbs = ORACLE_SAMPLE[args.workload]
+        wl.oracle_sample(oracle, 1, 1)
+        for _ in range(args.warmup):
+            wl.oracle_sample(oracle, 2, 1)
+        t0 = time.perf_counter()
+        work = 0.0
+        for _ in range(args.steps):
+            work += wl.oracle_sample(oracle, rows, nbs)
+        dt = time.perf_counter() - t0
+        v = round(work / dt / scale(wl), 6)
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": v, "unit": wl.unit,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt * 1e3 / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": wl.config(),
+            "cpu_baseline": {"value": v, "unit": wl.unit, "cores": oracle.num_threads(),
+                             "kind": "oracle",
+                             "sample": "per step: %d rows x %d 128-column blocks of the "
+                                       "workload with their online quantization" % (rows, nbs)},
+            "e2e": {"value": v, "unit": wl.unit, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+        }))
+        return
+
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        wl, elapsed_ms, per_kernel, clk, e2e, wall, dev_err = run_ours(args, rank, world,
+                                                                       local_rank)
+        if rank != 0:
+            return
+        peaks, peak_src = load_peaks()
+        value = world * wl.work_per_step() * args.steps / (elapsed_ms / 1e3) / scale(wl)
+        kernels = {}
+        for k, ms in per_kernel.items():
+            r = roofline_entry(wl, k, ms, peaks, peak_src)
+            kernels[k] = {"us": round(ms * 1e3, 2), "achieved": r["achieved"], "unit": r["unit"],
+                          "frac": r["frac"]}
+        dom = wl.dominant
+        roof = roofline_entry(wl, dom, per_kernel[dom], peaks, peak_src)
+        roof["traffic"] = recorded_traffic(dom, args.workload)
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": wl.unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(elapsed_ms / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate)",
+            "data": "synthetic (seeded, DeepSeek-V3 layer shapes)", "config": wl.config(),
+            "roofline": roof, "kernels": kernels,
+            "gpu_launches": len(wl.kernels) * args.steps,
+            "clocks": clk, "e2e": e2e, "device_error": dev_err,
+            "wall_s_timed_region": round(wall, 4),
+            "parallelism": "replicas (dp%d, no collective on the data path)" % world,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(args, wl_cls)
+        print(json.dumps(line))
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

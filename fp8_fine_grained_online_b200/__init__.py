@@ -1,0 +1,173 @@
+"""Fine-grained online FP8 (E4M3) quantization and block-scaled FP8 GEMM
+for NVIDIA B200 (sm_100a).
+
+Python binding of the C ABI declared in ``include/fp8fg.h``.  Each function
+below has the name of the C entry point it calls and only marshals
+arguments: it reads pointers, sizes and strides from ``torch.Tensor``
+objects (allocating outputs with torch when they are not given) and passes
+the current CUDA stream.  All computation happens in the CUDA library;
+importing this package fails if that library is not built.
+
+Method (codingmall.com "Kan du förklara rollen för FP8 precision i
+träningsprocessen för DeepSeek-V3"): activations are quantized in 1x128
+tiles and weights in 128x128 blocks, each with its own scale amax/448
+computed on every call, into E4M3; the FP8 GEMM promotes each 128-wide
+K chunk's tensor-core partial to FP32 after multiplying it by the two
+scales.
+"""
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import (FP8_IN_BF16, FP8_IN_FP32, FP8_OUT_BF16, FP8_OUT_FP32, LIB_PATH,
+                   STATUS_NAMES, Fp8Error)
+
+__all__ = [
+    "fp8_quantize_act_1x128", "fp8_quantize_weight_128x128", "fp8_blockscaled_gemm",
+    "fp8_grouped_gemm", "fp8_status_string", "fp8_get_device_error", "Fp8Error",
+    "LIB_PATH", "linear_forward", "e2e_linear_forward",
+]
+
+_L = _lib.lib
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _in_type(t):
+    if t.dtype == torch.bfloat16:
+        return FP8_IN_BF16
+    if t.dtype == torch.float32:
+        return FP8_IN_FP32
+    raise TypeError("inputs are bfloat16 or float32, got %s" % t.dtype)
+
+
+def _out_type(dtype):
+    if dtype == torch.bfloat16:
+        return FP8_OUT_BF16
+    if dtype == torch.float32:
+        return FP8_OUT_FP32
+    raise TypeError("outputs are bfloat16 or float32, got %s" % dtype)
+
+
+def _rowmajor(t, name):
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("%s must be a 2-D tensor with a contiguous last dimension" % name)
+
+
+def fp8_status_string(status):
+    return _L.fp8_status_string(int(status)).decode()
+
+
+def fp8_get_device_error(stream=None):
+    """Synchronize the stream, then read and clear the device error word."""
+    code = ctypes.c_int(0)
+    _lib.check(_L.fp8_get_device_error(_stream(stream), ctypes.byref(code)),
+               "fp8_get_device_error")
+    return code.value
+
+
+def fp8_quantize_act_1x128(x, q=None, sa=None, stream=None):
+    """x [M, K] (bf16/fp32, CUDA) -> (q uint8 [M, K] E4M3 codes, sa fp32 [M, K/128])."""
+    _rowmajor(x, "x")
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    if sa is None:
+        sa = torch.empty((M, K // 128), dtype=torch.float32, device=x.device)
+    _rowmajor(q, "q")
+    st = _L.fp8_quantize_act_1x128(_ptr(x), _in_type(x), M, K, x.stride(0), _ptr(q), q.stride(0),
+                                   _ptr(sa), sa.stride(0), sa.stride(1), _stream(stream))
+    _lib.check(st, "fp8_quantize_act_1x128")
+    return q, sa
+
+
+def fp8_quantize_weight_128x128(w, transpose_out=True, q=None, sb=None, stream=None):
+    """w [K, N] -> (q uint8 [N, K] if transpose_out else [K, N], sb fp32 [K/128, N/128])."""
+    _rowmajor(w, "w")
+    K, N = w.shape
+    if q is None:
+        shape = (N, K) if transpose_out else (K, N)
+        q = torch.empty(shape, dtype=torch.uint8, device=w.device)
+    if sb is None:
+        sb = torch.empty((K // 128, N // 128), dtype=torch.float32, device=w.device)
+    _rowmajor(q, "q")
+    st = _L.fp8_quantize_weight_128x128(_ptr(w), _in_type(w), K, N, w.stride(0), _ptr(q),
+                                        1 if transpose_out else 0, q.stride(0), _ptr(sb),
+                                        sb.stride(0), sb.stride(1), _stream(stream))
+    _lib.check(st, "fp8_quantize_weight_128x128")
+    return q, sb
+
+
+def fp8_blockscaled_gemm(a, sa, b, sb, out_dtype=torch.bfloat16, c=None, sb_kb_nb=True,
+                         stream=None):
+    """C [M, N] = block-scaled a [M, K] x b^T, b stored K-major [N, K].
+
+    sa is indexed [m, kb]; sb is indexed [kb, nb] (``sb_kb_nb``) or, when
+    False, stored [nb, kb] (the untransposed weight used for dgrad).
+    """
+    _rowmajor(a, "a")
+    _rowmajor(b, "b")
+    M, K = a.shape
+    N = b.shape[0]
+    if c is None:
+        c = torch.empty((M, N), dtype=out_dtype, device=a.device)
+    _rowmajor(c, "c")
+    sb_skb, sb_snb = (sb.stride(0), sb.stride(1)) if sb_kb_nb else (sb.stride(1), sb.stride(0))
+    st = _L.fp8_blockscaled_gemm(_ptr(a), a.stride(0), _ptr(sa), sa.stride(0), sa.stride(1),
+                                 _ptr(b), b.stride(0), 1, _ptr(sb), sb_skb, sb_snb, _ptr(c),
+                                 _out_type(c.dtype), c.stride(0), M, N, K, _stream(stream))
+    _lib.check(st, "fp8_blockscaled_gemm")
+    return c
+
+
+def fp8_grouped_gemm(a, sa, b, sb, offsets, out_dtype=torch.bfloat16, c=None, stream=None):
+    """MoE grouped GEMM: a [total_M, K] rows sorted by group, b [G, N, K],
+    sb [G, K/128, N/128], offsets int32 [G+1] on the device."""
+    _rowmajor(a, "a")
+    if b.dim() != 3 or b.stride(2) != 1 or b.stride(0) != b.shape[1] * b.stride(1):
+        raise ValueError("b must be [G, N, K] with K contiguous and experts contiguous")
+    total, K = a.shape
+    G, N, _ = b.shape
+    if c is None:
+        c = torch.empty((total, N), dtype=out_dtype, device=a.device)
+    _rowmajor(c, "c")
+    if offsets.dtype != torch.int32 or offsets.numel() != G + 1:
+        raise ValueError("offsets must be int32 [G+1]")
+    st = _L.fp8_grouped_gemm(_ptr(a), a.stride(0), _ptr(sa), sa.stride(0), sa.stride(1), _ptr(b),
+                             b.stride(1), _ptr(sb), sb.stride(0), sb.stride(1), sb.stride(2),
+                             _ptr(c), _out_type(c.dtype), c.stride(0), _ptr(offsets), G, total,
+                             N, K, _stream(stream))
+    _lib.check(st, "fp8_grouped_gemm")
+    return c
+
+
+def linear_forward(x, w, out_dtype=torch.bfloat16, stream=None):
+    """Online-quantized FP8 linear layer: y = x @ w with x [M, K], w [K, N].
+
+    Quantizes x in 1x128 tiles and w in 128x128 blocks (scales computed on
+    this call), then runs the block-scaled GEMM.  Three library calls.
+    """
+    qx, sx = fp8_quantize_act_1x128(x, stream=stream)
+    qw, sw = fp8_quantize_weight_128x128(w, transpose_out=True, stream=stream)
+    return fp8_blockscaled_gemm(qx, sx, qw, sw, out_dtype=out_dtype, stream=stream)
+
+
+def e2e_linear_forward(x_host, w_host, out_host=None, device="cuda", stream=None):
+    """End-to-end form of ``linear_forward`` on host tensors: copies x and w
+    (ideally pinned) to the device, runs the three library calls, and copies
+    y back into ``out_host`` (allocated pinned when not given)."""
+    x = x_host.to(device, non_blocking=True)
+    w = w_host.to(device, non_blocking=True)
+    y = linear_forward(x, w, out_dtype=torch.bfloat16, stream=stream)
+    if out_host is None:
+        out_host = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+    out_host.copy_(y, non_blocking=True)
+    return out_host

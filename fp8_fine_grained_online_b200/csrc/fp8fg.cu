@@ -1,0 +1,360 @@
+// fp8fg.cu -- C ABI of the library (declared in include/fp8fg.h): argument
+// validation, per-device capability checks, TMA descriptor encoding and
+// kernel launches.  Single translation unit: the kernels and the device
+// error word live in the headers included below.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/fp8fg.h"
+#include "gemm_kernels.cuh"
+#include "quant_kernels.cuh"
+
+namespace fp8fg {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    std::atomic<int> state{0};  // 0 unknown, 1 ok, 2 unsupported
+    int num_sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+// Current device must be compute capability 10.0 (B200, sm_100a code).
+fp8_status_t current_device(int* dev_out, int* sms_out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return FP8_ERR_DEVICE;
+    }
+    DeviceInfo& d = g_dev[dev];
+    int st = d.state.load(std::memory_order_acquire);
+    if (st == 0) {
+        std::lock_guard<std::mutex> lk(g_dev_mu);
+        st = d.state.load(std::memory_order_relaxed);
+        if (st == 0) {
+            int major = 0, minor = 0, sms = 0;
+            if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+                cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+                cudaGetLastError();
+                return FP8_ERR_CUDA;
+            }
+            bool ok = (major == 10 && minor == 0);
+            if (ok) {
+                // Opt the GEMM kernels into their shared-memory footprint.
+                const void* kernels[] = {
+                    reinterpret_cast<const void*>(&blockscaled_gemm_kernel<false, false>),
+                    reinterpret_cast<const void*>(&blockscaled_gemm_kernel<false, true>),
+                    reinterpret_cast<const void*>(&blockscaled_gemm_kernel<true, false>),
+                    reinterpret_cast<const void*>(&blockscaled_gemm_kernel<true, true>)};
+                for (const void* k : kernels) {
+                    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kGemmSmemBytes)) != cudaSuccess) {
+                        cudaGetLastError();
+                        return FP8_ERR_CUDA;
+                    }
+                }
+            }
+            d.num_sms = sms;
+            st = ok ? 1 : 2;
+            d.state.store(st, std::memory_order_release);
+        }
+    }
+    if (st != 1) return FP8_ERR_DEVICE;
+    *dev_out = dev;
+    *sms_out = d.num_sms;
+    return FP8_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        else
+            cudaGetLastError();
+    });
+    return g_encode;
+}
+
+// 2-D uint8 tensor [rows, cols] with row stride `ld` bytes, box
+// [box_rows, 128 bytes], 128-byte swizzle, zero fill out of bounds.
+bool make_operand_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                      uint64_t ld, uint32_t box_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {ld};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+inline fp8_status_t launch_status() {
+    return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+int elem_size_in(fp8_in_t t) { return t == FP8_IN_BF16 ? 2 : (t == FP8_IN_FP32 ? 4 : 0); }
+int elem_size_out(fp8_out_t t) { return t == FP8_OUT_BF16 ? 2 : (t == FP8_OUT_FP32 ? 4 : 0); }
+
+// Grid of resident-sized blocks, a multiple of the SM count.
+int64_t grid_for(int64_t work_blocks, int sms, int blocks_per_sm) {
+    const int64_t cap = static_cast<int64_t>(sms) * blocks_per_sm;
+    return work_blocks < cap ? work_blocks : cap;
+}
+
+// K == 0: the product is empty, C = 0.  Only c is used.
+fp8_status_t zero_output(void* c, fp8_out_t ct, int64_t ldc, int64_t rows, int64_t cols,
+                         cudaStream_t stream) {
+    const int oes = elem_size_out(ct);
+    if (!c) return FP8_ERR_NULL;
+    if (ldc < cols) return FP8_ERR_LAYOUT;
+    if (!aligned16(c) || (ldc * oes) % 16 != 0) return FP8_ERR_ALIGN;
+    int dev, sms;
+    fp8_status_t st = current_device(&dev, &sms);
+    if (st != FP8_OK) return st;
+    const int64_t grid = grid_for((rows * cols + 255) / 256, sms, 8);
+    if (ct == FP8_OUT_BF16)
+        zero_rows_kernel<__nv_bfloat16><<<static_cast<unsigned>(grid), 256, 0, stream>>>(
+            static_cast<__nv_bfloat16*>(c), rows, cols, ldc);
+    else
+        zero_rows_kernel<float><<<static_cast<unsigned>(grid), 256, 0, stream>>>(
+            static_cast<float*>(c), rows, cols, ldc);
+    return launch_status();
+}
+
+}  // namespace
+}  // namespace fp8fg
+
+using namespace fp8fg;
+
+extern "C" {
+
+const char* fp8_status_string(fp8_status_t s) {
+    switch (s) {
+        case FP8_OK: return "FP8_OK";
+        case FP8_ERR_NULL: return "FP8_ERR_NULL: a required pointer is NULL";
+        case FP8_ERR_SHAPE: return "FP8_ERR_SHAPE: bad size (negative, or not a multiple of 128)";
+        case FP8_ERR_ALIGN: return "FP8_ERR_ALIGN: pointer or leading dimension not 16-byte aligned";
+        case FP8_ERR_LAYOUT: return "FP8_ERR_LAYOUT: unsupported strides or operand orientation";
+        case FP8_ERR_DTYPE: return "FP8_ERR_DTYPE: unknown element type";
+        case FP8_ERR_DEVICE: return "FP8_ERR_DEVICE: current device is not an sm_100 (B200) GPU";
+        case FP8_ERR_CUDA: return "FP8_ERR_CUDA: a CUDA call failed";
+        case FP8_ERR_UNIMPLEMENTED: return "FP8_ERR_UNIMPLEMENTED";
+        case FP8_ERR_DEVICE_TIMEOUT: return "FP8_ERR_DEVICE_TIMEOUT: a kernel gave up waiting";
+    }
+    return "unknown fp8_status_t";
+}
+
+fp8_status_t fp8_quantize_act_1x128(const void* x, fp8_in_t x_type, int64_t M, int64_t K,
+                                    int64_t ldx, uint8_t* q, int64_t ldq, float* sa,
+                                    int64_t sa_stride_m, int64_t sa_stride_kb,
+                                    fp8_stream_t stream) {
+    const int es = elem_size_in(x_type);
+    if (es == 0) return FP8_ERR_DTYPE;
+    if (M < 0 || K < 0 || K % 128 != 0) return FP8_ERR_SHAPE;
+    if (M == 0 || K == 0) return FP8_OK;
+    if (!x || !q || !sa) return FP8_ERR_NULL;
+    if (ldx < K || ldq < K || sa_stride_m < 0 || sa_stride_kb < 0) return FP8_ERR_LAYOUT;
+    if (!aligned16(x) || (ldx * es) % 16 != 0 || !aligned16(q) || ldq % 16 != 0 || !aligned4(sa))
+        return FP8_ERR_ALIGN;
+    int dev, sms;
+    fp8_status_t st = current_device(&dev, &sms);
+    if (st != FP8_OK) return st;
+
+    const int64_t nkb = K / 128;
+    const int64_t tiles = M * nkb;
+    const int64_t per_block = 16 * kActUnroll;
+    const int64_t grid = grid_for((tiles + per_block - 1) / per_block, sms, 8);
+    if (x_type == FP8_IN_BF16)
+        quant_act_1x128_kernel<uint16_t><<<static_cast<unsigned>(grid), kActThreads, 0, stream>>>(
+            static_cast<const uint16_t*>(x), M, nkb, ldx, q, ldq, sa, sa_stride_m, sa_stride_kb);
+    else
+        quant_act_1x128_kernel<float><<<static_cast<unsigned>(grid), kActThreads, 0, stream>>>(
+            static_cast<const float*>(x), M, nkb, ldx, q, ldq, sa, sa_stride_m, sa_stride_kb);
+    return launch_status();
+}
+
+fp8_status_t fp8_quantize_weight_128x128(const void* w, fp8_in_t w_type, int64_t K, int64_t N,
+                                         int64_t ldw, uint8_t* q, int transpose_out,
+                                         int64_t ldq, float* sb, int64_t sb_stride_kb,
+                                         int64_t sb_stride_nb, fp8_stream_t stream) {
+    const int es = elem_size_in(w_type);
+    if (es == 0) return FP8_ERR_DTYPE;
+    if (K < 0 || N < 0 || K % 128 != 0 || N % 128 != 0) return FP8_ERR_SHAPE;
+    if (K == 0 || N == 0) return FP8_OK;
+    if (!w || !q || !sb) return FP8_ERR_NULL;
+    if (ldw < N || ldq < (transpose_out ? K : N) || sb_stride_kb < 0 || sb_stride_nb < 0)
+        return FP8_ERR_LAYOUT;
+    if (!aligned16(w) || (ldw * es) % 16 != 0 || !aligned16(q) || ldq % 16 != 0 || !aligned4(sb))
+        return FP8_ERR_ALIGN;
+    int dev, sms;
+    fp8_status_t st = current_device(&dev, &sms);
+    if (st != FP8_OK) return st;
+
+    const int64_t nkb = K / 128, nnb = N / 128;
+    const int64_t grid = grid_for(nkb * nnb, sms, 8);
+    if (w_type == FP8_IN_BF16)
+        quant_weight_128x128_kernel<uint16_t><<<static_cast<unsigned>(grid), kWThreads, 0, stream>>>(
+            static_cast<const uint16_t*>(w), nkb, nnb, ldw, q, transpose_out ? 1 : 0, ldq, sb,
+            sb_stride_kb, sb_stride_nb);
+    else
+        quant_weight_128x128_kernel<float><<<static_cast<unsigned>(grid), kWThreads, 0, stream>>>(
+            static_cast<const float*>(w), nkb, nnb, ldw, q, transpose_out ? 1 : 0, ldq, sb,
+            sb_stride_kb, sb_stride_nb);
+    return launch_status();
+}
+
+static fp8_status_t check_gemm_common(const uint8_t* a, int64_t lda, const float* sa,
+                                      int64_t sa_sm, int64_t sa_skb, const uint8_t* b, int64_t ldb,
+                                      const float* sb, int64_t sb_skb, int64_t sb_snb, void* c,
+                                      fp8_out_t ct, int64_t ldc, int64_t N, int64_t K) {
+    const int oes = elem_size_out(ct);
+    if (oes == 0) return FP8_ERR_DTYPE;
+    if (!a || !sa || !b || !sb || !c) return FP8_ERR_NULL;
+    if (lda < K || ldb < K || ldc < N || sa_sm < 0 || sa_skb < 0 || sb_skb < 0 || sb_snb < 0)
+        return FP8_ERR_LAYOUT;
+    if (!aligned16(a) || lda % 16 != 0 || !aligned16(b) || ldb % 16 != 0 || !aligned16(c) ||
+        (ldc * oes) % 16 != 0 || !aligned4(sa) || !aligned4(sb))
+        return FP8_ERR_ALIGN;
+    if (K / 128 > INT32_MAX / 2 || N > (static_cast<int64_t>(1) << 31)) return FP8_ERR_SHAPE;
+    return FP8_OK;
+}
+
+fp8_status_t fp8_blockscaled_gemm(const uint8_t* a, int64_t lda, const float* sa,
+                                  int64_t sa_stride_m, int64_t sa_stride_kb, const uint8_t* b,
+                                  int64_t ldb, int b_kmajor, const float* sb,
+                                  int64_t sb_stride_kb, int64_t sb_stride_nb, void* c,
+                                  fp8_out_t c_type, int64_t ldc, int64_t M, int64_t N, int64_t K,
+                                  fp8_stream_t stream) {
+    if (elem_size_out(c_type) == 0) return FP8_ERR_DTYPE;
+    if (M < 0 || N < 0 || K < 0 || N % 128 != 0 || K % 128 != 0) return FP8_ERR_SHAPE;
+    if (M == 0 || N == 0) return FP8_OK;
+    if (!b_kmajor) return FP8_ERR_LAYOUT;
+    if (K == 0) return zero_output(c, c_type, ldc, M, N, stream);
+    fp8_status_t st = check_gemm_common(a, lda, sa, sa_stride_m, sa_stride_kb, b, ldb, sb,
+                                        sb_stride_kb, sb_stride_nb, c, c_type, ldc, N, K);
+    if (st != FP8_OK) return st;
+    const int64_t num_mt = (M + kBM - 1) / kBM, num_nt = (N + kBN - 1) / kBN;
+    if (num_mt * num_nt > INT32_MAX || M > INT32_MAX) return FP8_ERR_SHAPE;
+    int dev, sms;
+    st = current_device(&dev, &sms);
+    if (st != FP8_OK) return st;
+
+    CUtensorMap tmA, tmB;
+    const uint64_t kcols = static_cast<uint64_t>(K);
+    if (!make_operand_map(&tmA, a, static_cast<uint64_t>(M), kcols, static_cast<uint64_t>(lda), kBM) ||
+        !make_operand_map(&tmB, b, static_cast<uint64_t>(N), kcols, static_cast<uint64_t>(ldb), kBN))
+        return FP8_ERR_CUDA;
+
+    GemmParams p{};
+    p.sa = sa; p.sa_sm = sa_stride_m; p.sa_skb = sa_stride_kb;
+    p.sb = sb; p.sb_sg = 0; p.sb_skb = sb_stride_kb; p.sb_snb = sb_stride_nb;
+    p.c = c; p.ldc = ldc; p.M = M; p.N = N;
+    p.nkb = static_cast<int>(K / 128);
+    p.num_mt = static_cast<int>(num_mt);
+    p.num_nt = static_cast<int>(num_nt);
+    p.band_m = 16;
+    p.offsets = nullptr; p.G = 1;
+    const int64_t grid = grid_for(num_mt * num_nt, sms, 1);
+    if (c_type == FP8_OUT_BF16)
+        blockscaled_gemm_kernel<false, true>
+            <<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, stream>>>(tmA, tmB, p);
+    else
+        blockscaled_gemm_kernel<false, false>
+            <<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, stream>>>(tmA, tmB, p);
+    return launch_status();
+}
+
+fp8_status_t fp8_grouped_gemm(const uint8_t* a, int64_t lda, const float* sa,
+                              int64_t sa_stride_m, int64_t sa_stride_kb, const uint8_t* b,
+                              int64_t ldb, const float* sb, int64_t sb_stride_g,
+                              int64_t sb_stride_kb, int64_t sb_stride_nb, void* c,
+                              fp8_out_t c_type, int64_t ldc, const int32_t* offsets, int G,
+                              int64_t total_M, int64_t N, int64_t K, fp8_stream_t stream) {
+    if (elem_size_out(c_type) == 0) return FP8_ERR_DTYPE;
+    if (G < 1 || G > kMaxGroups || total_M < 0 || N < 0 || K < 0 || N % 128 != 0 || K % 128 != 0)
+        return FP8_ERR_SHAPE;
+    if (total_M == 0 || N == 0) return FP8_OK;
+    if (K == 0) return zero_output(c, c_type, ldc, total_M, N, stream);
+    if (!offsets) return FP8_ERR_NULL;
+    if (!aligned4(offsets)) return FP8_ERR_ALIGN;
+    if (sb_stride_g < 0) return FP8_ERR_LAYOUT;
+    fp8_status_t st = check_gemm_common(a, lda, sa, sa_stride_m, sa_stride_kb, b, ldb, sb,
+                                        sb_stride_kb, sb_stride_nb, c, c_type, ldc, N, K);
+    if (st != FP8_OK) return st;
+    const int64_t num_nt = (N + kBN - 1) / kBN;
+    const int64_t max_mt = total_M / kBM + G;  // sum over groups of ceil(rows_g / 128)
+    if (total_M > INT32_MAX || max_mt * num_nt > INT32_MAX ||
+        static_cast<int64_t>(G) * N > INT32_MAX)
+        return FP8_ERR_SHAPE;
+    int dev, sms;
+    st = current_device(&dev, &sms);
+    if (st != FP8_OK) return st;
+
+    CUtensorMap tmA, tmB;
+    const uint64_t kcols = static_cast<uint64_t>(K);
+    if (!make_operand_map(&tmA, a, static_cast<uint64_t>(total_M), kcols, static_cast<uint64_t>(lda), kBM) ||
+        !make_operand_map(&tmB, b, static_cast<uint64_t>(G) * static_cast<uint64_t>(N), kcols,
+                          static_cast<uint64_t>(ldb), kBN))
+        return FP8_ERR_CUDA;
+
+    GemmParams p{};
+    p.sa = sa; p.sa_sm = sa_stride_m; p.sa_skb = sa_stride_kb;
+    p.sb = sb; p.sb_sg = sb_stride_g; p.sb_skb = sb_stride_kb; p.sb_snb = sb_stride_nb;
+    p.c = c; p.ldc = ldc; p.M = total_M; p.N = N;
+    p.nkb = static_cast<int>(K / 128);
+    p.num_mt = 0;
+    p.num_nt = static_cast<int>(num_nt);
+    p.band_m = 1;
+    p.offsets = offsets; p.G = G;
+    const int64_t grid = grid_for(max_mt * num_nt, sms, 1);
+    if (c_type == FP8_OUT_BF16)
+        blockscaled_gemm_kernel<true, true>
+            <<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, stream>>>(tmA, tmB, p);
+    else
+        blockscaled_gemm_kernel<true, false>
+            <<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, stream>>>(tmA, tmB, p);
+    return launch_status();
+}
+
+fp8_status_t fp8_get_device_error(fp8_stream_t stream, fp8_status_t* code) {
+    if (!code) return FP8_ERR_NULL;
+    int dev, sms;
+    fp8_status_t st = current_device(&dev, &sms);
+    if (st != FP8_OK) return st;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) {
+        cudaGetLastError();
+        return FP8_ERR_CUDA;
+    }
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof v) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero) != cudaSuccess) {
+        cudaGetLastError();
+        return FP8_ERR_CUDA;
+    }
+    *code = static_cast<fp8_status_t>(v);
+    return FP8_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,433 @@
+// gemm_kernels.cuh -- block-scaled FP8 GEMM on sm_100a tensor cores
+// (tcgen05 UMMA, TMEM accumulators, TMA operand loads), dense and MoE-grouped.
+//
+//   C[m, n] = sum_kb sa[m, kb] * sb[kb, n/128] * P_kb[m, n]
+//   P_kb    = the tensor-core product of one 128-wide K chunk of E4M3 codes
+//
+// The promotion interval is one 128-wide chunk, the scaling unit of both
+// operands (codingmall.com "Kan du förklara rollen för FP8 precision i
+// träningsprocessen för DeepSeek-V3", "Ökad ackumuleringsprecision": the
+// tensor-core partial sums are promoted to FP32 registers at fixed
+// intervals; "Finkornig kvantisering" for the 1x128 / 128x128 scales).
+//
+// Structure (one persistent CTA per SM, 320 threads):
+//   warp 0      TMA producer: A tile 128x128 B and B tile 256x128 B per chunk
+//               into a 4-stage shared-memory ring (128-byte swizzle).
+//   warp 1      TMEM owner and MMA issuer: per chunk, 4 x UMMA
+//               (M=128, N=256, K=32) into one of two TMEM partial buffers
+//               (2 x 256 columns), then commits to the ring's "empty"
+//               barrier and the buffer's "full" barrier.
+//   warps 2-9   epilogue: warp w reads TMEM lanes 32*(w%4).. and columns
+//               128*((w-2)/4).., scales the chunk partial by sa*sb and adds
+//               it to 128 FP32 accumulators per thread (one output row,
+//               128 columns); at tile end converts and stores the row.
+// Double-buffered TMEM lets the MMA of chunk kb+1 run while the epilogue
+// promotes chunk kb.
+//
+// Every mbarrier wait is bounded (kWaitLimitNs); on timeout the kernel
+// records FP8_ERR_DEVICE_TIMEOUT in the device error word, all roles stop,
+// in-flight copies and MMAs are waited for (bounded), TMEM is released and
+// the kernel returns.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "sm100_ptx.cuh"
+
+namespace fp8fg {
+
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kBK = 128;  // one scale chunk = 128 bytes of E4M3 per row
+constexpr int kStages = 4;
+// 12 warps = 3 warpgroups.  Warps 0-7 (warpgroups 0-1) are the epilogue;
+// warpgroup 2 holds the TMA producer (warp 8), the MMA issuer / TMEM owner
+// (warp 9) and two idle warps.  Registers at launch: 384 x 168; warpgroup 2
+// drops to kCtrlRegs and warpgroups 0-1 rise to kEpiRegs:
+// 128 x 40 + 256 x 232 = 64512 = 384 x 168.
+constexpr int kGemmThreads = 384;
+constexpr int kEpiWarps = 8;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kSchedWarp = 10;
+constexpr int kCtrlRegs = 40;
+constexpr int kEpiRegs = 232;
+static_assert(128 * kCtrlRegs + 256 * kEpiRegs <= kGemmThreads * 168, "register split");
+constexpr int kABytes = kBM * kBK;  // 16 KB
+constexpr int kBBytes = kBN * kBK;  // 32 KB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kTmemCols = 512;      // 2 partial buffers x 256 FP32 columns
+constexpr int kMaxGroups = 1024;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
+
+// Status codes recorded in the device error word (values of fp8_status_t).
+constexpr unsigned kDevErrShape = 2;
+constexpr unsigned kDevErrTimeout = 9;
+
+// Device error word; read and cleared by fp8_get_device_error().
+__device__ unsigned int g_device_error = 0;
+
+__device__ __forceinline__ void record_device_error(unsigned code) {
+    atomicCAS(&g_device_error, 0u, code);
+}
+
+struct GemmParams {
+    const float* sa;
+    int64_t sa_sm, sa_skb;
+    const float* sb;
+    int64_t sb_sg, sb_skb, sb_snb;
+    void* c;
+    int64_t ldc;
+    int64_t M;       // dense: rows; grouped: total rows
+    int64_t N;
+    int nkb;         // K / 128
+    int num_nt;      // ceil(N / kBN)
+    int num_mt;      // dense only: ceil(M / kBM)
+    int band_m;      // dense raster: m-tiles per band
+    const int32_t* offsets;  // grouped only: [G + 1]
+    int G;
+};
+
+// Shared-memory layout after the 1024-aligned operand ring.
+struct GemmSmemTail {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint32_t tmem_base;
+    int abort_flag;
+    int total_tiles;
+    int pad;
+    int grp_prefix[kMaxGroups + 1];  // grouped: tiles before group g
+    int grp_lo[kMaxGroups];          // grouped: first row of group g
+    int grp_hi[kMaxGroups];          // grouped: one past its last row (clamped)
+};
+
+constexpr size_t kGemmSmemBytes = 1024 /* alignment slack */ + kStages * kStageBytes +
+                                  sizeof(GemmSmemTail);
+
+struct TileCoord {
+    int64_t m0;       // first row of the tile (global row index)
+    int64_t row_end;  // rows >= row_end are not part of this tile's problem
+    int64_t n0;       // first column
+    int g;            // group (0 for dense)
+};
+
+// Wait for phase `parity` of `bar` to complete; false if this CTA aborted or
+// the wait ran past kWaitLimitNs (which aborts the CTA).
+__device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity,
+                                             volatile int* abort_flag) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(a, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            record_device_error(kDevErrTimeout);
+            return false;
+        }
+    }
+}
+
+// Same, ignoring the abort flag: used on the abort path to drain copies
+// and MMAs this thread issued, so that no async write outlives the CTA.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+    const uint32_t a = smem_u32(bar);
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(a, parity)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            record_device_error(kDevErrTimeout);
+            return;
+        }
+    }
+}
+
+template <bool kGrouped>
+__device__ __forceinline__ TileCoord decode_tile(int t, const GemmParams& p,
+                                                 const GemmSmemTail* tail) {
+    TileCoord tc;
+    if (!kGrouped) {
+        // Bands of band_m m-tiles; inside a band, m runs fastest so that the
+        // CTAs of one wave share both A rows and B columns through L2.
+        const int per_band = p.band_m * p.num_nt;
+        const int band = t / per_band;
+        const int within = t - band * per_band;
+        const int bm0 = band * p.band_m;
+        const int bm = min(p.band_m, p.num_mt - bm0);
+        const int nt = within / bm;
+        const int mt = bm0 + (within - nt * bm);
+        tc.m0 = static_cast<int64_t>(mt) * kBM;
+        tc.row_end = p.M;
+        tc.n0 = static_cast<int64_t>(nt) * kBN;
+        tc.g = 0;
+    } else {
+        // Group g owns tiles [grp_prefix[g], grp_prefix[g+1]).
+        int lo = 0, hi = p.G;  // find the last g with grp_prefix[g] <= t
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (tail->grp_prefix[mid] <= t) lo = mid; else hi = mid;
+        }
+        const int g = lo;
+        const int local = t - tail->grp_prefix[g];
+        const int rows = tail->grp_hi[g] - tail->grp_lo[g];
+        const int nmt = (rows + kBM - 1) / kBM;
+        const int nt = local / nmt;
+        const int mt = local - nt * nmt;  // m fastest: neighbours share B tiles
+        tc.m0 = tail->grp_lo[g] + static_cast<int64_t>(mt) * kBM;
+        tc.row_end = tail->grp_hi[g];
+        tc.n0 = static_cast<int64_t>(nt) * kBN;
+        tc.g = g;
+    }
+    return tc;
+}
+
+template <bool kGrouped, bool kOutBf16>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    blockscaled_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                            const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+    uint8_t* sA = smem;                         // kStages x 16 KB
+    uint8_t* sB = smem + kStages * kABytes;     // kStages x 32 KB
+    GemmSmemTail* tail = reinterpret_cast<GemmSmemTail*>(smem + kStages * kStageBytes);
+    volatile int* abort_flag = &tail->abort_flag;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (warp == kProducerWarp && lane == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&tail->full[s], 1);
+            mbar_init(&tail->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tail->tfull[b], 1);
+            mbar_init(&tail->tempty[b], kEpiWarps);
+        }
+        tail->abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(&tail->tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    if (kGrouped && warp == kSchedWarp) {
+        // Tile table from the device offsets: group g has ceil(rows_g/128)
+        // m-tiles times num_nt n-tiles.  Invalid offsets give empty groups.
+        int carry = 0;
+        for (int base = 0; base < p.G; base += 32) {
+            const int g = base + lane;
+            int tiles = 0;
+            if (g < p.G) {
+                int64_t lo = p.offsets[g];
+                int64_t hi = p.offsets[g + 1];
+                if (lo < 0 || hi < lo) {
+                    record_device_error(kDevErrShape);
+                    lo = hi = 0;
+                }
+                lo = lo < p.M ? lo : p.M;
+                hi = hi < p.M ? hi : p.M;
+                tail->grp_lo[g] = static_cast<int>(lo);
+                tail->grp_hi[g] = static_cast<int>(hi);
+                tiles = static_cast<int>((hi - lo + kBM - 1) / kBM) * p.num_nt;
+            }
+            int incl = tiles;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+                if (lane >= off) incl += y;
+            }
+            if (g < p.G) tail->grp_prefix[g + 1] = carry + incl;
+            carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        }
+        if (lane == 0) {
+            tail->grp_prefix[0] = 0;
+            tail->total_tiles = carry;
+        }
+    } else if (!kGrouped && warp == kSchedWarp && lane == 0) {
+        tail->total_tiles = p.num_mt * p.num_nt;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem_base = tail->tmem_base;
+    const int total_tiles = tail->total_tiles;
+    const int nkb = p.nkb;
+
+    if (warp >= kEpiWarps) {
+        // Control warpgroup (producer, MMA, two idle warps): few registers.
+        setmaxnreg_dec<kCtrlRegs>();
+        if (warp == kProducerWarp && lane == 0) {
+            // ------------------------------------------------ TMA producer
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued_mask = 0, last_parity = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+                const TileCoord tc = decode_tile<kGrouped>(t, p, tail);
+                const int32_t a_row = static_cast<int32_t>(tc.m0);
+                const int32_t b_row = static_cast<int32_t>(tc.g * p.N + tc.n0);
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!bounded_wait(&tail->empty[stage], phase ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&tail->full[stage], kStageBytes);
+                    tma_load_2d(sA + stage * kABytes, &tmA, &tail->full[stage], kb * kBK, a_row);
+                    tma_load_2d(sB + stage * kBBytes, &tmB, &tail->full[stage], kb * kBK, b_row);
+                    issued_mask |= 1u << stage;
+                    last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                for (int s = 0; s < kStages; ++s)
+                    if (issued_mask & (1u << s)) drain_wait(&tail->full[s], (last_parity >> s) & 1u);
+            }
+        } else if (warp == kMmaWarp && lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            constexpr uint32_t idesc = idesc_e4m3_f32(kBM, kBN);
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t chunk = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+                for (int kb = 0; kb < nkb; ++kb) {
+                    const uint32_t buf = chunk & 1u;
+                    const uint32_t use = chunk >> 1;
+                    if (!bounded_wait(&tail->tempty[buf], (use & 1u) ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (!bounded_wait(&tail->full[stage], phase, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(sA + stage * kABytes));
+                    const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(sB + stage * kBBytes));
+                    const uint32_t d = tmem_base + buf * kBN;
+#pragma unroll
+                    for (int k = 0; k < kBK / 32; ++k)  // 32 bytes of K per MMA = +2 in addr>>4
+                        umma_f8f6f4(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+                    umma_commit(&tail->empty[stage]);
+                    umma_commit(&tail->tfull[buf]);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                    ++chunk;
+                }
+            }
+            if (!ok && chunk > 0) {
+                const uint32_t last = chunk - 1;
+                drain_wait(&tail->tfull[last & 1u], (last >> 1) & 1u);
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue warps 0-7
+        setmaxnreg_inc<kEpiRegs>();
+        const int q = warp & 3;            // TMEM lane quarter of this warp
+        const int h = warp >> 2;           // column half of the 256-wide tile
+        const int r = q * 32 + lane;       // row within the tile
+        const uint32_t t_lane = static_cast<uint32_t>(q * 32) << 16;
+        uint32_t chunk = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+            const TileCoord tc = decode_tile<kGrouped>(t, p, tail);
+            const int64_t row = tc.m0 + r;
+            const bool row_ok = row < tc.row_end;
+            const int64_t col0 = tc.n0 + h * 128;
+            const bool col_ok = col0 < p.N;
+            const float* sa_row = p.sa + (row_ok ? row : 0) * p.sa_sm;
+            const float* sb_col = p.sb + tc.g * p.sb_sg + (col_ok ? col0 / 128 : 0) * p.sb_snb;
+
+            float acc[128];
+#pragma unroll
+            for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+            float sa_next = (row_ok && nkb > 0) ? __ldg(sa_row) : 0.0f;
+            float sb_next = (col_ok && nkb > 0) ? __ldg(sb_col) : 0.0f;
+
+            for (int kb = 0; kb < nkb; ++kb) {
+                const float scale = sa_next * sb_next;
+                if (kb + 1 < nkb) {
+                    sa_next = row_ok ? __ldg(sa_row + (kb + 1) * p.sa_skb) : 0.0f;
+                    sb_next = col_ok ? __ldg(sb_col + (kb + 1) * p.sb_skb) : 0.0f;
+                }
+                const uint32_t buf = chunk & 1u;
+                const uint32_t use = chunk >> 1;
+                if (!bounded_wait(&tail->tfull[buf], use & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t taddr = tmem_base + t_lane + buf * kBN + h * 128;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    uint32_t part0[32], part1[32];
+                    tmem_ld_32x32b_x32(taddr + j * 64, part0);
+                    tmem_ld_32x32b_x32(taddr + j * 64 + 32, part1);
+                    tmem_wait_ld();
+                    if (j == 1) {
+                        // Both halves of this warp's slice are in registers:
+                        // hand the TMEM buffer back to the MMA warp.
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&tail->tempty[buf]);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        acc[j * 64 + i] = fmaf(scale, __uint_as_float(part0[i]), acc[j * 64 + i]);
+                        acc[j * 64 + 32 + i] =
+                            fmaf(scale, __uint_as_float(part1[i]), acc[j * 64 + 32 + i]);
+                    }
+                }
+                ++chunk;
+            }
+            if (!ok) break;
+            if (row_ok && col_ok) {
+                if (kOutBf16) {
+                    __nv_bfloat16* out =
+                        reinterpret_cast<__nv_bfloat16*>(p.c) + row * p.ldc + col0;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const __nv_bfloat162 b2 =
+                                __floats2bfloat162_rn(acc[j * 8 + 2 * e], acc[j * 8 + 2 * e + 1]);
+                            w[e] = *reinterpret_cast<const uint32_t*>(&b2);
+                        }
+                        reinterpret_cast<uint4*>(out)[j] = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                } else {
+                    float* out = reinterpret_cast<float*>(p.c) + row * p.ldc + col0;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        reinterpret_cast<float4*>(out)[j] =
+                            make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kMmaWarp) tmem_dealloc(tmem_base, kTmemCols);
+}
+
+}  // namespace fp8fg

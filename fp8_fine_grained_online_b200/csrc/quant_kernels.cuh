@@ -1,0 +1,225 @@
+// quant_kernels.cuh -- online fine-grained E4M3 quantization kernels.
+//
+// Both kernels compute, per tile / block, scale = amax / 448 (IEEE fp32
+// division, 1 when zero) and code = E4M3_RNE_satfinite(x / scale) with one
+// IEEE fp32 division per element (codingmall.com "Kan du förklara rollen
+// för FP8 precision i träningsprocessen för DeepSeek-V3": "Finkornig
+// kvantisering", "Online-kvantisering"; holysheep.ai "FP8 混精度训练
+// DeepSeek 671B" (zh), 2.2).  They are HBM-bound: each input element is
+// read once with 16-byte loads and each code written once.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "sm100_ptx.cuh"
+
+namespace fp8fg {
+
+constexpr float kE4M3Max = 448.0f;
+
+template <typename T>
+struct InVec;  // 8 consecutive input elements, loaded with 16-byte accesses
+
+template <>
+struct InVec<uint16_t> {  // bf16 bit patterns
+    static __device__ __forceinline__ void load(const uint16_t* p, float (&v)[8]) {
+        const uint4 w = __ldcs(reinterpret_cast<const uint4*>(p));
+        const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[2 * i] = __uint_as_float(u[i] << 16);           // exact bf16 -> fp32
+            v[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
+        }
+    }
+};
+
+template <>
+struct InVec<float> {
+    static __device__ __forceinline__ void load(const float* p, float (&v)[8]) {
+        const float4 a = __ldcs(reinterpret_cast<const float4*>(p));
+        const float4 b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+};
+
+__device__ __forceinline__ float scale_from_amax(float amax) {
+    float s = __fdiv_rn(amax, kE4M3Max);
+    return s == 0.0f ? 1.0f : s;
+}
+
+// 8 values / scale -> 8 E4M3 codes packed little-endian in a uint2.
+__device__ __forceinline__ uint2 encode8(const float (&v)[8], float s) {
+    float d[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) d[i] = __fdiv_rn(v[i], s);
+    uint2 r;
+    r.x = cvt_e4m3x2(d[0], d[1]) | (cvt_e4m3x2(d[2], d[3]) << 16);
+    r.y = cvt_e4m3x2(d[4], d[5]) | (cvt_e4m3x2(d[6], d[7]) << 16);
+    return r;
+}
+
+// ---------------------------------------------------------------------------
+// 1x128 activation tiles.  A half-warp owns one tile: lane l of the half
+// loads elements [8l, 8l+8) of it, the tile amax is a 16-lane shuffle
+// reduction, and each lane stores 8 codes.  A block of 256 threads handles
+// 16 * kActUnroll consecutive tiles per step, issuing all loads first.
+// ---------------------------------------------------------------------------
+constexpr int kActThreads = 256;
+constexpr int kActUnroll = 4;
+
+template <typename T>
+__global__ void __launch_bounds__(kActThreads)
+    quant_act_1x128_kernel(const T* __restrict__ x, int64_t M, int64_t nkb, int64_t ldx,
+                           uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sa,
+                           int64_t sa_sm, int64_t sa_skb) {
+    const int hl = threadIdx.x & 15;          // lane within the half-warp
+    const int hw = threadIdx.x >> 4;          // half-warp within the block (0..15)
+    const int64_t total = M * nkb;
+    const int64_t step = static_cast<int64_t>(gridDim.x) * (16 * kActUnroll);
+
+    for (int64_t base = static_cast<int64_t>(blockIdx.x) * (16 * kActUnroll); base < total;
+         base += step) {
+        float v[kActUnroll][8];
+        int64_t row[kActUnroll], kb[kActUnroll];
+#pragma unroll
+        for (int u = 0; u < kActUnroll; ++u) {
+            const int64_t t = base + u * 16 + hw;
+            row[u] = t / nkb;
+            kb[u] = t - row[u] * nkb;
+            if (t < total) {
+                InVec<T>::load(x + row[u] * ldx + kb[u] * 128 + hl * 8, v[u]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[u][i] = 0.0f;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kActUnroll; ++u) {
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[u][i]));  // NaN skipped
+#pragma unroll
+            for (int off = 8; off > 0; off >>= 1)
+                amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+            const float s = scale_from_amax(amax);
+            const int64_t t = base + u * 16 + hw;
+            if (t < total) {
+                const uint2 codes = encode8(v[u], s);
+                __stcs(reinterpret_cast<uint2*>(q + row[u] * ldq + kb[u] * 128 + hl * 8), codes);
+                if (hl == 0) sa[row[u] * sa_sm + kb[u] * sa_skb] = s;
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 128x128 weight blocks.  One block of 256 threads owns one 128x128 block:
+// thread (kq = tid/16, c = tid%16) holds rows {4kq..4kq+3, 64+4kq..64+4kq+3}
+// and columns [8c, 8c+8).  The block amax is reduced through shared memory,
+// then codes are written either directly ([K, N]) or through a shared
+// transpose buffer ([N, K]).
+// ---------------------------------------------------------------------------
+constexpr int kWThreads = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(kWThreads)
+    quant_weight_128x128_kernel(const T* __restrict__ w, int64_t nkb, int64_t nnb, int64_t ldw,
+                                uint8_t* __restrict__ q, int transpose_out, int64_t ldq,
+                                float* __restrict__ sb, int64_t sb_skb, int64_t sb_snb) {
+    __shared__ float red[kWThreads / 32];
+    __shared__ uint32_t tbuf[128][33];  // [n][k/4] words, one padding word per row
+
+    const int tid = threadIdx.x;
+    const int c = tid & 15;
+    const int kq = tid >> 4;
+    const int64_t nblocks = nkb * nnb;
+
+    for (int64_t blk = blockIdx.x; blk < nblocks; blk += gridDim.x) {
+        const int64_t kb = blk / nnb;
+        const int64_t nb = blk - kb * nnb;
+        const T* src = w + (kb * 128) * ldw + nb * 128 + c * 8;
+
+        float v[8][8];  // [row slot][column]
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int k = (r >> 2) * 64 + kq * 4 + (r & 3);
+            InVec<T>::load(src + k * ldw, v[r]);
+        }
+        float amax = 0.0f;
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[r][i]));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+        if ((tid & 31) == 0) red[tid >> 5] = amax;
+        __syncthreads();
+        amax = red[0];
+#pragma unroll
+        for (int i = 1; i < kWThreads / 32; ++i) amax = fmaxf(amax, red[i]);
+        const float s = scale_from_amax(amax);
+        if (tid == 0) sb[kb * sb_skb + nb * sb_snb] = s;
+
+        uint2 codes[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) codes[r] = encode8(v[r], s);
+
+        if (!transpose_out) {
+            uint8_t* dst = q + (kb * 128) * ldq + nb * 128 + c * 8;
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const int k = (r >> 2) * 64 + kq * 4 + (r & 3);
+                __stcs(reinterpret_cast<uint2*>(dst + k * ldq), codes[r]);
+            }
+        } else {
+            // Gather, per column n, the 4 codes of rows 4kq..4kq+3 (and the
+            // +64 group) into one word: tbuf[n][k/4].
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    uint32_t word = 0;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint2 cj = codes[h * 4 + j];
+                        const uint32_t half = (i < 4) ? cj.x : cj.y;
+                        word |= ((half >> ((i & 3) * 8)) & 0xFFu) << (8 * j);
+                    }
+                    tbuf[c * 8 + i][h * 16 + kq] = word;
+                }
+            }
+            __syncthreads();
+            // Thread (n = tid/2, part = tid%2) writes 64 codes of row n of q^T.
+            const int n = tid >> 1;
+            const int part = tid & 1;
+            uint8_t* dst = q + (nb * 128 + n) * ldq + kb * 128 + part * 64;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint4 o;
+                o.x = tbuf[n][part * 16 + j * 4 + 0];
+                o.y = tbuf[n][part * 16 + j * 4 + 1];
+                o.z = tbuf[n][part * 16 + j * 4 + 2];
+                o.w = tbuf[n][part * 16 + j * 4 + 3];
+                __stcs(reinterpret_cast<uint4*>(dst) + j, o);
+            }
+        }
+        __syncthreads();  // red[] and tbuf[] are reused by the next block
+    }
+}
+
+// C = 0 for a GEMM with an empty contraction (K == 0).
+template <typename T>
+__global__ void __launch_bounds__(256)
+    zero_rows_kernel(T* __restrict__ c, int64_t rows, int64_t cols, int64_t ldc) {
+    const int64_t total = rows * cols;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t r = i / cols;
+        c[r * ldc + (i - r * cols)] = T(0);
+    }
+}
+
+}  // namespace fp8fg

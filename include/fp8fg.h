@@ -1,0 +1,204 @@
+/*
+ * fp8fg.h -- C ABI of the fine-grained online FP8 library for NVIDIA B200
+ * (sm_100a): online 1x128 / 128x128 E4M3 quantization and the block-scaled
+ * FP8 GEMM (dense and MoE-grouped) that consumes its output.
+ *
+ * The method these calls implement is the FP8 mixed-precision scheme of
+ * DeepSeek-V3 as described in
+ *   [KB] codingmall.com knowledge base, "Kan du förklara rollen för FP8
+ *        precision i träningsprocessen för DeepSeek-V3"
+ *        (sections "Mixed Precision Framework", "Finkornig kvantisering",
+ *        "Online-kvantisering", "Ökad ackumuleringsprecision",
+ *        "Unified E4M3 Format"), and
+ *   [HS] holysheep.ai, "FP8 混精度训练 DeepSeek 671B" (Chinese edition),
+ *        section "2.2 细粒度量化实现" (scale = amax / 448, divide, cast to
+ *        E4M3; dequantize = code value x scale).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - E4M3 is the "e4m3fn" encoding: bias 7, no infinities, NaN = S.1111.111,
+ *    largest finite magnitude 448.  Codes are stored as raw bytes (uint8).
+ *  - Quantization rounds x / scale (one IEEE fp32 division) to the nearest
+ *    E4M3 value, ties to even, saturating to +-448; scale = amax / 448 in
+ *    IEEE fp32, replaced by 1 when it is zero.  Results are bit-identical
+ *    to that definition.
+ *  - Pointers named as device pointers must be device (or managed) memory
+ *    of the CURRENT CUDA device; the caller owns every buffer.  The library
+ *    allocates no device memory and keeps no per-call state.
+ *  - Every call is asynchronous on `stream` (NULL = the legacy default
+ *    stream).  Nothing synchronizes, prints, aborts or throws.
+ *  - Matrices are row-major with a leading dimension (`ld*`, in ELEMENTS)
+ *    between consecutive rows; the innermost dimension is contiguous.
+ *  - Argument errors are reported synchronously by the return value, before
+ *    any work is queued.  A problem with zero rows (or zero columns) is a
+ *    valid no-op that returns FP8_OK; its pointers may then be NULL.
+ *  - Requires a compute-capability 10.0 device (B200); any other device
+ *    gives FP8_ERR_DEVICE.
+ */
+#ifndef FP8FG_H
+#define FP8FG_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define FP8FG_API __attribute__((visibility("default")))
+#else
+#define FP8FG_API
+#endif
+
+struct CUstream_st;                       /* cudaStream_t == struct CUstream_st* */
+typedef struct CUstream_st* fp8_stream_t;
+
+typedef enum fp8_status {
+    FP8_OK = 0,
+    FP8_ERR_NULL = 1,          /* a required pointer is NULL                          */
+    FP8_ERR_SHAPE = 2,         /* negative size, or a dimension not a multiple of 128 */
+    FP8_ERR_ALIGN = 3,         /* a pointer or leading dimension breaks 16-byte rules */
+    FP8_ERR_LAYOUT = 4,        /* strides/orientation this call does not support      */
+    FP8_ERR_DTYPE = 5,         /* unknown element-type enum value                     */
+    FP8_ERR_DEVICE = 6,        /* no current device, or it is not sm_100             */
+    FP8_ERR_CUDA = 7,          /* a CUDA runtime/driver call failed                   */
+    FP8_ERR_UNIMPLEMENTED = 8,
+    FP8_ERR_DEVICE_TIMEOUT = 9 /* (from fp8_get_device_error) a kernel gave up waiting */
+} fp8_status_t;
+
+typedef enum fp8_in_type { FP8_IN_BF16 = 0, FP8_IN_FP32 = 1 } fp8_in_t;
+typedef enum fp8_out_type { FP8_OUT_FP32 = 0, FP8_OUT_BF16 = 1 } fp8_out_t;
+
+/*
+ * fp8_quantize_act_1x128 -- online fine-grained activation quantization.
+ * [KB] "Finkornig kvantisering" (activations in 1x128 tiles, each scaled on
+ * its own) and "Online-kvantisering" (scale from the current values on every
+ * call); [HS] 2.2 (scale = amax / 448, x / scale cast to E4M3).
+ *
+ * For every row m and every 128-wide tile kb of x [M, K]:
+ *     amax        = max_k |x[m, k]|           (k in the tile)
+ *     sa[m, kb]   = amax / 448   (1 if that is 0)
+ *     q[m, k]     = E4M3_RNE_satfinite(x[m, k] / sa[m, kb])
+ *
+ *  x      device, [M, ldx] elements of type x_type (bf16 or fp32); 16-byte
+ *         aligned, ldx * sizeof(elem) a multiple of 16, ldx >= K.
+ *  M, K   M >= 0 any value; K >= 0 and a multiple of 128.
+ *  q      device, [M, ldq] bytes written (codes); 16-byte aligned,
+ *         ldq a multiple of 16, ldq >= K.
+ *  sa     device fp32; sa[m * sa_stride_m + kb * sa_stride_kb] written for
+ *         0 <= kb < K/128.  Any non-negative strides (e.g. [M, K/128]
+ *         row-major: sa_stride_m = K/128, sa_stride_kb = 1).
+ *  Errors: FP8_ERR_NULL, FP8_ERR_SHAPE, FP8_ERR_ALIGN, FP8_ERR_DTYPE,
+ *          FP8_ERR_LAYOUT (negative stride), FP8_ERR_DEVICE, FP8_ERR_CUDA.
+ */
+FP8FG_API fp8_status_t fp8_quantize_act_1x128(const void* x, fp8_in_t x_type, int64_t M, int64_t K,
+                                    int64_t ldx, uint8_t* q, int64_t ldq, float* sa,
+                                    int64_t sa_stride_m, int64_t sa_stride_kb,
+                                    fp8_stream_t stream);
+
+/*
+ * fp8_quantize_weight_128x128 -- online fine-grained weight quantization.
+ * [KB] "Finkornig kvantisering" (weights in 128x128 blocks, each scaled on
+ * its own), "Online-kvantisering"; [HS] 2.2.
+ *
+ * For every 128x128 block (kb, nb) of w [K, N]:
+ *     sb[kb, nb] = amax(block) / 448   (1 if that is 0)
+ *     code(k, n) = E4M3_RNE_satfinite(w[k, n] / sb[kb, nb])
+ * written to q[k * ldq + n] (transpose_out == 0, q is [K, N]) or
+ * q[n * ldq + k] (transpose_out == 1, q is [N, K]: the K-major operand the
+ * forward GEMM reads).  The untransposed [K, N] form is itself the K-major
+ * operand of the transposed product (dgrad, dX = dY W^T), with sb read as
+ * [nb][kb]; one quantization of w serves both products.
+ *
+ *  w      device, [K, ldw] elements of w_type; 16-byte aligned,
+ *         ldw * sizeof(elem) a multiple of 16, ldw >= N.
+ *  K, N   multiples of 128 (>= 0).
+ *  q      device bytes, 16-byte aligned, ldq a multiple of 16,
+ *         ldq >= N (transpose_out == 0) or >= K (transpose_out == 1).
+ *  sb     device fp32, sb[kb * sb_stride_kb + nb * sb_stride_nb].
+ */
+FP8FG_API fp8_status_t fp8_quantize_weight_128x128(const void* w, fp8_in_t w_type, int64_t K,
+                                         int64_t N, int64_t ldw, uint8_t* q,
+                                         int transpose_out, int64_t ldq, float* sb,
+                                         int64_t sb_stride_kb, int64_t sb_stride_nb,
+                                         fp8_stream_t stream);
+
+/*
+ * fp8_blockscaled_gemm -- FP8 GEMM with per-chunk FP32 promotion.
+ * [KB] "Mixed Precision Framework" (the GEMMs run in FP8), "Ökad
+ * ackumuleringsprecision" (tensor-core partial sums promoted to FP32
+ * registers at fixed intervals), "Unified E4M3 Format"; [HS] 2.2 dequantize.
+ *
+ *     C[m, n] = sum_kb  sa[m, kb] * sb[kb, n/128] * P_kb[m, n]
+ *     P_kb[m, n] = sum_{k in chunk kb} E4M3(a[m, k]) * E4M3(b(n, k))
+ *
+ * The promotion interval is one 128-wide K chunk (the scaling unit): each
+ * chunk's tensor-core partial P_kb is scaled and added into an FP32
+ * accumulator.  C is written as fp32 or bf16 (round to nearest even).
+ *
+ *  a      device codes [M, lda] (K-major), 16-byte aligned, lda % 16 == 0,
+ *         lda >= K.
+ *  sa     device fp32, sa[m * sa_stride_m + kb * sa_stride_kb].
+ *  b      device codes; b_kmajor must be 1: b is [N, ldb], b(n, k) =
+ *         b[n * ldb + k], 16-byte aligned, ldb % 16 == 0, ldb >= K.
+ *         (b_kmajor == 0 gives FP8_ERR_LAYOUT; quantize with
+ *         transpose_out = 1 to obtain the K-major operand.)
+ *  sb     device fp32, sb[kb * sb_stride_kb + nb * sb_stride_nb].
+ *  c      device [M, ldc] of c_type, 16-byte aligned,
+ *         ldc * sizeof(elem) % 16 == 0, ldc >= N.
+ *  M      >= 0, any value (rows beyond M are never written).
+ *  N, K   multiples of 128 (>= 0).  K == 0 writes C = 0.
+ */
+FP8FG_API fp8_status_t fp8_blockscaled_gemm(const uint8_t* a, int64_t lda, const float* sa,
+                                  int64_t sa_stride_m, int64_t sa_stride_kb,
+                                  const uint8_t* b, int64_t ldb, int b_kmajor,
+                                  const float* sb, int64_t sb_stride_kb,
+                                  int64_t sb_stride_nb, void* c, fp8_out_t c_type,
+                                  int64_t ldc, int64_t M, int64_t N, int64_t K,
+                                  fp8_stream_t stream);
+
+/*
+ * fp8_grouped_gemm -- the block-scaled GEMM over MoE expert groups.
+ * Same arithmetic as fp8_blockscaled_gemm ([KB] "Mixed Precision
+ * Framework", "Ökad ackumuleringsprecision"), applied per expert g to the
+ * rows [offsets[g], offsets[g+1]) of a (rows sorted by expert):
+ *
+ *     C[m, n] = sum_kb sa[m, kb] * sb_g[kb, n/128] * P_kb[m, n]   with B_g
+ *
+ *  a, sa  as in fp8_blockscaled_gemm, total_M rows.
+ *  b      device codes [G][N][ldb] (each expert K-major, experts contiguous:
+ *         expert g starts at b + g * N * ldb); alignment as above.
+ *  sb     device fp32, sb[g * sb_stride_g + kb * sb_stride_kb + nb * sb_stride_nb].
+ *  c      device [total_M, ldc] of c_type.
+ *  offsets device int32 [G + 1]: offsets[0] = 0, non-decreasing,
+ *         offsets[G] = total_M.  Read on the device (no host sync).  A
+ *         decreasing pair makes that group empty and records
+ *         FP8_ERR_SHAPE in the device error word; rows at or beyond
+ *         total_M are never read or written.
+ *  G      1 <= G <= 1024.
+ */
+FP8FG_API fp8_status_t fp8_grouped_gemm(const uint8_t* a, int64_t lda, const float* sa,
+                              int64_t sa_stride_m, int64_t sa_stride_kb, const uint8_t* b,
+                              int64_t ldb, const float* sb, int64_t sb_stride_g,
+                              int64_t sb_stride_kb, int64_t sb_stride_nb, void* c,
+                              fp8_out_t c_type, int64_t ldc, const int32_t* offsets, int G,
+                              int64_t total_M, int64_t N, int64_t K, fp8_stream_t stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+FP8FG_API const char* fp8_status_string(fp8_status_t status);
+
+/*
+ * fp8_get_device_error -- synchronizes `stream`, then reads and clears the
+ * current device's error word.  Kernels record into it when a bounded wait
+ * gives up (FP8_ERR_DEVICE_TIMEOUT; the kernel then stops early and its
+ * outputs are undefined) or when the grouped GEMM meets invalid offsets
+ * (FP8_ERR_SHAPE).  *code receives the recorded status (FP8_OK if none).
+ * Returns FP8_ERR_CUDA if the synchronization or the read fails.
+ */
+FP8FG_API fp8_status_t fp8_get_device_error(fp8_stream_t stream, fp8_status_t* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8FG_H */

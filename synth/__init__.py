@@ -168,7 +168,8 @@ def moe_inputs(device="cpu", tokens=8192, experts=256, topk=8, hidden=7168, inte
     Returns dict with: x_routed bf16 [tokens*topk, hidden] (rows sorted by
     expert), offsets int32 [experts+1], h_down bf16 [tokens*topk, inter]
     (input of the down projection, N(0,1)), and when ``with_weights``:
-    w_gate_up bf16 [experts, hidden, 2*inter], w_down bf16 [experts, inter, hidden].
+    w_gate_up bf16 [experts, hidden, 2*inter], w_down bf16 [experts, inter, hidden]
+    (built expert by expert with ``moe_expert_weight``).
     """
     c = MOE.config_id
     x = act_input(tokens, hidden, 1.0, 1e-3, 100.0, c, device)
@@ -176,6 +177,21 @@ def moe_inputs(device="cpu", tokens=8192, experts=256, topk=8, hidden=7168, inte
     out = dict(x_routed=x[token_of].contiguous(), offsets=offsets, token_of=token_of)
     out["h_down"] = normal((tokens * topk, inter), 1.0, seed_for(c, 3), device)
     if with_weights:
-        out["w_gate_up"] = normal((experts, hidden, 2 * inter), 0.02, seed_for(c, 8), device)
-        out["w_down"] = normal((experts, inter, hidden), 0.02, seed_for(c, 9), device)
+        out["w_gate_up"] = torch.stack([moe_expert_weight(e, "gate_up", device, hidden, inter)
+                                        for e in range(experts)])
+        out["w_down"] = torch.stack([moe_expert_weight(e, "down", device, hidden, inter)
+                                     for e in range(experts)])
     return out
+
+
+def moe_expert_weight(e, which, device="cpu", hidden=7168, inter=2048):
+    """Expert e's weight, bf16 N(0, 0.02): "gate_up" [hidden, 2*inter] (gate
+    and up projections side by side along N) or "down" [inter, hidden]."""
+    c = MOE.config_id
+    if which == "gate_up":
+        shape, tid = (hidden, 2 * inter), 8
+    elif which == "down":
+        shape, tid = (inter, hidden), 9
+    else:
+        raise ValueError(which)
+    return normal(shape, 0.02, seed_for(c, tid) + (e + 1) * 1_000_003, device)

@@ -1,0 +1,151 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry
+point ``include/fp8fg.h`` declares, the Python binding uses the same names,
+and argument validation answers synchronously before any CUDA work.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8fg.h")
+
+
+def declared_functions():
+    text = open(HEADER, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp8_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from fp8_fine_grained_online_b200 import _lib
+    return _lib.lib
+
+
+def test_header_declares_the_four_entry_points():
+    names = declared_functions()
+    for n in ("fp8_quantize_act_1x128", "fp8_quantize_weight_128x128", "fp8_blockscaled_gemm",
+              "fp8_grouped_gemm", "fp8_status_string", "fp8_get_device_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_binding_covers_every_declared_symbol():
+    import fp8_fine_grained_online_b200 as fp8
+    from fp8_fine_grained_online_b200 import _lib
+    for name in declared_functions():
+        assert name in _lib.SIGNATURES, name
+        assert callable(getattr(fp8, name)), name
+
+
+def test_library_exports_nothing_else(L):
+    """Hidden visibility: only the C ABI is exported."""
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", L._name], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert exported == set(declared_functions())
+
+
+def test_status_strings(L):
+    for code in range(10):
+        s = L.fp8_status_string(code).decode()
+        assert s.startswith("FP8_")
+    assert L.fp8_status_string(99).decode() == "unknown fp8_status_t"
+
+
+P = ctypes.c_void_p
+A16 = P(0x10000)          # an aligned, never-dereferenced address
+A8 = P(0x10008)
+
+
+def act(L, x=A16, xt=0, M=4, K=128, ldx=128, q=A16, ldq=128, sa=A16, sm=1, skb=4):
+    return L.fp8_quantize_act_1x128(x, xt, M, K, ldx, q, ldq, sa, sm, skb, None)
+
+
+def test_act_argument_errors(L):
+    assert act(L, xt=7) == 5                       # DTYPE
+    assert act(L, K=100, ldx=128) == 2             # SHAPE: K % 128
+    assert act(L, M=-1) == 2
+    assert act(L, M=0, x=None, q=None, sa=None) == 0   # empty: no-op
+    assert act(L, K=0, x=None, q=None, sa=None) == 0
+    assert act(L, x=None) == 1                     # NULL
+    assert act(L, sa=None) == 1
+    assert act(L, ldx=64) == 4                     # LAYOUT: ldx < K
+    assert act(L, skb=-1) == 4
+    assert act(L, x=A8) == 3                       # ALIGN
+    assert act(L, q=A8) == 3
+    assert act(L, ldx=132) == 3                    # 132 bf16 = 264 B, not 16-B multiple
+    assert act(L, ldq=136) == 3
+    assert act(L, sa=P(0x10002)) == 3
+
+
+def test_weight_argument_errors(L):
+    def w(**kw):
+        a = dict(w=A16, wt=0, K=128, N=256, ldw=256, q=A16, tr=1, ldq=128, sb=A16, skb=2, snb=1)
+        a.update(kw)
+        return L.fp8_quantize_weight_128x128(a["w"], a["wt"], a["K"], a["N"], a["ldw"], a["q"],
+                                             a["tr"], a["ldq"], a["sb"], a["skb"], a["snb"], None)
+    assert w(N=200, ldw=256) == 2
+    assert w(K=0, w=None) == 0
+    assert w(q=None) == 1
+    assert w(tr=1, ldq=64) == 4                    # transposed q is [N, K]: ldq >= K
+    assert w(tr=0, ldq=128) == 4                   # [K, N]: ldq >= N
+    assert w(w=A8) == 3
+    assert w(wt=3) == 5
+
+
+def gemm(L, **kw):
+    a = dict(a=A16, lda=256, sa=A16, sam=1, sakb=128, b=A16, ldb=256, bk=1, sb=A16, sbkb=2,
+             sbnb=1, c=A16, ct=1, ldc=256, M=128, N=256, K=256)
+    a.update(kw)
+    return L.fp8_blockscaled_gemm(a["a"], a["lda"], a["sa"], a["sam"], a["sakb"], a["b"],
+                                  a["ldb"], a["bk"], a["sb"], a["sbkb"], a["sbnb"], a["c"],
+                                  a["ct"], a["ldc"], a["M"], a["N"], a["K"], None)
+
+
+def test_gemm_argument_errors(L):
+    assert gemm(L, ct=4) == 5
+    assert gemm(L, K=200) == 2
+    assert gemm(L, N=100) == 2
+    assert gemm(L, M=0, a=None) == 0
+    assert gemm(L, bk=0) == 4                      # only K-major B
+    assert gemm(L, sb=None) == 1
+    assert gemm(L, lda=128) == 4
+    assert gemm(L, a=A8) == 3
+    assert gemm(L, ldb=264) == 3
+    assert gemm(L, ldc=260) == 3                   # 260 bf16 = 520 B
+
+
+def test_grouped_argument_errors(L):
+    def g(**kw):
+        a = dict(a=A16, lda=256, sa=A16, sam=1, sakb=64, b=A16, ldb=256, sb=A16, sbg=4,
+                 sbkb=2, sbnb=1, c=A16, ct=1, ldc=256, off=A16, G=4, M=64, N=256, K=256)
+        a.update(kw)
+        return L.fp8_grouped_gemm(a["a"], a["lda"], a["sa"], a["sam"], a["sakb"], a["b"],
+                                  a["ldb"], a["sb"], a["sbg"], a["sbkb"], a["sbnb"], a["c"],
+                                  a["ct"], a["ldc"], a["off"], a["G"], a["M"], a["N"], a["K"],
+                                  None)
+    assert g(G=0) == 2
+    assert g(G=1025) == 2
+    assert g(M=0) == 0
+    assert g(off=None) == 1
+    assert g(off=P(0x10001)) == 3
+    assert g(sbg=-1) == 4
+
+
+def test_valid_arguments_without_gpu_report_device_error(L):
+    """With every argument valid, the next check is the device: no GPU here."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is visible")
+    assert act(L) == 6
+    assert gemm(L) == 6
+    code = ctypes.c_int(0)
+    assert L.fp8_get_device_error(None, ctypes.byref(code)) == 6

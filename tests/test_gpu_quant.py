@@ -1,0 +1,149 @@
+"""GPU parity of the online quantization kernels against the oracle:
+codes and scales bit-identical, called through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from _util import assert_codes_equal, assert_scales_equal, np_u8, to_oracle
+
+pytestmark = pytest.mark.gpu
+
+
+def act(M, K, dtype, seed, std=1.0, outliers=1e-2):
+    return synth.act_input(M, K, std, outliers, 100.0, 7, "cpu", dtype, tensor_id=seed)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("M,K", [(1, 128), (3, 256), (130, 384), (257, 1024), (1000, 7168),
+                                 (77, 2048)])
+def test_act_quant_bit_exact(cuda_lib, orc, M, K, dtype):
+    x = act(M, K, dtype, M + K)
+    q, sa = cuda_lib.fp8_quantize_act_1x128(x.cuda())
+    qo, sao = orc.quantize_act_1x128(to_oracle(x))
+    assert_codes_equal(np_u8(q), qo)
+    assert_scales_equal(sa.cpu().numpy(), sao)
+
+
+def test_act_quant_strided_layouts(cuda_lib, orc):
+    """ldx > K, ldq > K and column-major ([K/128, M]) scales."""
+    M, K = 200, 512
+    big = act(M, 768, torch.bfloat16, 3).cuda()
+    x = big[:, 128:128 + K]
+    qbuf = torch.full((M, 640), 0xAB, dtype=torch.uint8, device="cuda")
+    q = qbuf[:, 64:64 + K]
+    sa_t = torch.full((K // 128, M), -1.0, device="cuda")
+    cuda_lib.fp8_quantize_act_1x128(x, q=q, sa=sa_t.t())
+    qo, sao = orc.quantize_act_1x128(to_oracle(x))
+    assert_codes_equal(np_u8(q), qo)
+    assert_scales_equal(sa_t.t().cpu().numpy(), sao)
+    untouched = np_u8(qbuf)
+    assert np.all(untouched[:, :64] == 0xAB) and np.all(untouched[:, 64 + K:] == 0xAB)
+
+
+def test_act_quant_special_values(cuda_lib, orc):
+    x = torch.randn(8, 512) * 3
+    x[0, :128] = 0.0                               # zero tile -> scale 1
+    x[0, 128:256] = -0.0
+    x[1, :128] = 1e-42                             # subnormal fp32 amax: amax/448 underflows
+    x[1, 5] = -1e-42
+    x[2, :128] = torch.tensor(2.0 ** -130)         # subnormal scale, no underflow
+    x[3, 130] = 3.0e38                             # huge amax
+    x[4, 256:384] = 448.0                          # all at the maximum
+    x[5, 384:] = torch.linspace(-1e-3, 1e-3, 128)
+    for dtype in (torch.float32, torch.bfloat16):
+        xd = x.to(dtype)
+        q, sa = cuda_lib.fp8_quantize_act_1x128(xd.cuda())
+        qo, sao = orc.quantize_act_1x128(to_oracle(xd))
+        assert_codes_equal(np_u8(q), qo)
+        assert_scales_equal(sa.cpu().numpy(), sao)
+
+
+def test_cvt_rounding_matches_oracle_encoder(cuda_lib, orc):
+    """Every tile holds 448 so its scale is exactly 1 and code = E4M3(x):
+    checks the hardware conversion against the oracle's nearest-value
+    encoder on random values and on every midpoint +-1 ulp."""
+    dec = orc.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+    mids = ((dec[:-1] + dec[1:]) / 2).astype(np.float32)
+    special = np.concatenate([mids, np.nextafter(mids, np.float32(0)),
+                              np.nextafter(mids, np.float32(np.inf)), dec.astype(np.float32)])
+    special = np.concatenate([special, -special])
+    rng = np.random.default_rng(42)
+    rand = (np.exp2(rng.uniform(-14, np.log2(448), 2_000_000)) *
+            rng.choice([-1, 1], 2_000_000)).astype(np.float32)
+    vals = np.concatenate([special, rand])
+    n_rows = (len(vals) + 126) // 127
+    tiles = np.zeros((n_rows, 128), dtype=np.float32)
+    tiles[:, 0] = 448.0
+    tiles[:, 1:].flat[:len(vals)] = vals
+    x = torch.from_numpy(tiles)
+    q, sa = cuda_lib.fp8_quantize_act_1x128(x.cuda())
+    assert torch.all(sa == 1.0)
+    assert_codes_equal(np_u8(q), orc.e4m3_encode(tiles))
+
+
+def test_act_quant_nan_element_smoke(cuda_lib, orc):
+    """Out of contract: a NaN element is skipped by amax and encodes to NaN."""
+    x = torch.randn(2, 256)
+    x[1, 17] = float("nan")
+    q, sa = cuda_lib.fp8_quantize_act_1x128(x.cuda())
+    qo, sao = orc.quantize_act_1x128(x.numpy())
+    g = np_u8(q)
+    assert (g[1, 17] & 0x7F) == 0x7F
+    g[1, 17] = qo[1, 17]
+    assert_codes_equal(g, qo)
+    assert_scales_equal(sa.cpu().numpy(), sao)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("K,N", [(128, 128), (256, 384), (384, 256), (1024, 2048)])
+@pytest.mark.parametrize("transpose", [False, True])
+def test_weight_quant_bit_exact(cuda_lib, orc, K, N, dtype, transpose):
+    w = synth.normal((K, N), 0.02, 1000 + K + N, "cpu", dtype)
+    synth.scale_outliers(w, 1e-3, 100.0, 77)
+    q, sb = cuda_lib.fp8_quantize_weight_128x128(w.cuda(), transpose_out=transpose)
+    qo, sbo = orc.quantize_weight_128x128(to_oracle(w), transpose_out=transpose)
+    assert_codes_equal(np_u8(q), qo)
+    assert_scales_equal(sb.cpu().numpy(), sbo)
+
+
+def test_weight_quant_zero_and_strided(cuda_lib, orc):
+    K, N = 256, 384
+    big = synth.normal((K, 512), 0.02, 5, "cpu", torch.float32)
+    big[:128, :128] = 0.0
+    w = big[:, 64:64 + N].cuda()
+    sbT = torch.zeros((N // 128, K // 128), device="cuda")
+    for transpose in (False, True):
+        q, _ = cuda_lib.fp8_quantize_weight_128x128(w, transpose_out=transpose, sb=sbT.t())
+        qo, sbo = orc.quantize_weight_128x128(to_oracle(w), transpose_out=transpose)
+        assert_codes_equal(np_u8(q), qo)
+        assert_scales_equal(sbT.t().cpu().numpy(), sbo)
+        assert sbo[0, 0] == 1.0
+
+
+# ---------------------------------------------------------------- full sizes
+
+def _sample_rows(M, n, seed):
+    rng = np.random.default_rng(seed)
+    return np.unique(np.concatenate([[0, M - 1], rng.integers(0, M, n)]))
+
+
+@pytest.mark.slow
+def test_quant_bandwidth_workload_sampled(cuda_lib, orc):
+    """Activation [8192x7168] and weight [7168x18432] bf16, N(0, 0.02) with
+    0.1% outliers x100, quantized as the bench does; sampled rows and
+    blocks compared bit for bit with the oracle."""
+    x, w = synth.quant_inputs("cuda")
+    q, sa = cuda_lib.fp8_quantize_act_1x128(x)
+    qw, sb = cuda_lib.fp8_quantize_weight_128x128(w, transpose_out=True)
+    torch.cuda.synchronize()
+    rows = _sample_rows(8192, 96, 1)
+    qo, sao = orc.quantize_act_1x128(to_oracle(x[torch.from_numpy(rows).cuda()]))
+    assert_codes_equal(np_u8(q[torch.from_numpy(rows).cuda()]), qo)
+    assert_scales_equal(sa[torch.from_numpy(rows).cuda()].cpu().numpy(), sao)
+    rng = np.random.default_rng(2)
+    for kb, nb in list(zip(rng.integers(0, 56, 24), rng.integers(0, 144, 24))) + [(55, 143)]:
+        blk = w[kb * 128:(kb + 1) * 128, nb * 128:(nb + 1) * 128]
+        qo, sbo = orc.quantize_weight_128x128(to_oracle(blk), transpose_out=True)
+        assert_codes_equal(np_u8(qw[nb * 128:(nb + 1) * 128, kb * 128:(kb + 1) * 128]), qo)
+        assert_scales_equal(sb[kb:kb + 1, nb:nb + 1].cpu().numpy(), sbo)
