@@ -186,12 +186,26 @@ fp8_status_t fp8_quantize_act_1x128(const void* x, fp8_in_t x_type, int64_t M, i
     const int64_t tiles = M * nkb;
     const int64_t per_block = 16 * kActUnroll;
     const int64_t grid = grid_for((tiles + per_block - 1) / per_block, sms, 8);
-    if (x_type == FP8_IN_BF16)
-        quant_act_1x128_kernel<uint16_t><<<static_cast<unsigned>(grid), kActThreads, 0, stream>>>(
-            static_cast<const uint16_t*>(x), M, nkb, ldx, q, ldq, sa, sa_stride_m, sa_stride_kb);
-    else
-        quant_act_1x128_kernel<float><<<static_cast<unsigned>(grid), kActThreads, 0, stream>>>(
-            static_cast<const float*>(x), M, nkb, ldx, q, ldq, sa, sa_stride_m, sa_stride_kb);
+    const bool small = tiles + per_block < (static_cast<int64_t>(1) << 31);
+    const FastDivU31 fd = FastDivU31::make(small ? static_cast<uint32_t>(nkb) : 1u);
+    const unsigned g = static_cast<unsigned>(grid);
+    if (x_type == FP8_IN_BF16) {
+        const uint16_t* xs = static_cast<const uint16_t*>(x);
+        if (small)
+            quant_act_1x128_kernel<uint16_t, true><<<g, kActThreads, 0, stream>>>(
+                xs, M, nkb, fd, ldx, q, ldq, sa, sa_stride_m, sa_stride_kb);
+        else
+            quant_act_1x128_kernel<uint16_t, false><<<g, kActThreads, 0, stream>>>(
+                xs, M, nkb, fd, ldx, q, ldq, sa, sa_stride_m, sa_stride_kb);
+    } else {
+        const float* xs = static_cast<const float*>(x);
+        if (small)
+            quant_act_1x128_kernel<float, true><<<g, kActThreads, 0, stream>>>(
+                xs, M, nkb, fd, ldx, q, ldq, sa, sa_stride_m, sa_stride_kb);
+        else
+            quant_act_1x128_kernel<float, false><<<g, kActThreads, 0, stream>>>(
+                xs, M, nkb, fd, ldx, q, ldq, sa, sa_stride_m, sa_stride_kb);
+    }
     return launch_status();
 }
 

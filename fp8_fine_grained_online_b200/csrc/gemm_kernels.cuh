@@ -186,6 +186,15 @@ __device__ __forceinline__ TileCoord decode_tile(int t, const GemmParams& p,
     return tc;
 }
 
+// acc[kOff .. kOff+32) += s * P (32 FP32 partials from TMEM), packed FMAs.
+template <int kOff>
+__device__ __forceinline__ void promote32(float (&acc)[128], const uint32_t (&part)[32], float s) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 2)
+        ffma2_scalar(acc[kOff + i], acc[kOff + i + 1], s, __uint_as_float(part[i]),
+                     __uint_as_float(part[i + 1]));
+}
+
 template <bool kGrouped, bool kOutBf16>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     blockscaled_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -361,6 +370,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             float sa_next = (row_ok && nkb > 0) ? __ldg(sa_row) : 0.0f;
             float sb_next = (col_ok && nkb > 0) ? __ldg(sb_col) : 0.0f;
 
+            // Software pipeline over 32-column batches of this warp's 128-column
+            // slice: the TMEM load of the next batch (also across chunk
+            // boundaries) is in flight while the current one is promoted.
+            uint32_t pa[32], pb[32];
+            if (nkb > 0) {
+                if (!bounded_wait(&tail->tfull[chunk & 1u], (chunk >> 1) & 1u, abort_flag)) break;
+                tc_fence_after();
+                tmem_ld_32x32b_x32(tmem_base + t_lane + (chunk & 1u) * kBN + h * 128, pa);
+            }
             for (int kb = 0; kb < nkb; ++kb) {
                 const float scale = sa_next * sb_next;
                 if (kb + 1 < nkb) {
@@ -368,34 +386,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     sb_next = col_ok ? __ldg(sb_col + (kb + 1) * p.sb_skb) : 0.0f;
                 }
                 const uint32_t buf = chunk & 1u;
-                const uint32_t use = chunk >> 1;
-                if (!bounded_wait(&tail->tfull[buf], use & 1u, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
                 const uint32_t taddr = tmem_base + t_lane + buf * kBN + h * 128;
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    uint32_t part0[32], part1[32];
-                    tmem_ld_32x32b_x32(taddr + j * 64, part0);
-                    tmem_ld_32x32b_x32(taddr + j * 64 + 32, part1);
-                    tmem_wait_ld();
-                    if (j == 1) {
-                        // Both halves of this warp's slice are in registers:
-                        // hand the TMEM buffer back to the MMA warp.
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&tail->tempty[buf]);
-                    }
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        acc[j * 64 + i] = fmaf(scale, __uint_as_float(part0[i]), acc[j * 64 + i]);
-                        acc[j * 64 + 32 + i] =
-                            fmaf(scale, __uint_as_float(part1[i]), acc[j * 64 + 32 + i]);
-                    }
-                }
+                tmem_wait_ld_dep(pa);
+                tmem_ld_32x32b_x32(taddr + 32, pb);
+                promote32<0>(acc, pa, scale);
+                tmem_wait_ld_dep(pb);
+                tmem_ld_32x32b_x32(taddr + 64, pa);
+                promote32<32>(acc, pb, scale);
+                tmem_wait_ld_dep(pa);
+                tmem_ld_32x32b_x32(taddr + 96, pb);
+                promote32<64>(acc, pa, scale);
+                tmem_wait_ld_dep(pb);
+                // This warp's slice of the chunk is in registers: hand the TMEM
+                // buffer back to the MMA warp.
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tail->tempty[buf]);
                 ++chunk;
+                if (kb + 1 < nkb) {
+                    if (!bounded_wait(&tail->tfull[chunk & 1u], (chunk >> 1) & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    tmem_ld_32x32b_x32(tmem_base + t_lane + (chunk & 1u) * kBN + h * 128, pa);
+                }
+                promote32<96>(acc, pb, scale);
             }
             if (!ok) break;
             if (row_ok && col_ok) {

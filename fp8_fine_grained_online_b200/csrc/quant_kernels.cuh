@@ -49,16 +49,76 @@ __device__ __forceinline__ float scale_from_amax(float amax) {
     return s == 0.0f ? 1.0f : s;
 }
 
-// 8 values / scale -> 8 E4M3 codes packed little-endian in a uint2.
-__device__ __forceinline__ uint2 encode8(const float (&v)[8], float s) {
-    float d[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) d[i] = __fdiv_rn(v[i], s);
-    uint2 r;
-    r.x = cvt_e4m3x2(d[0], d[1]) | (cvt_e4m3x2(d[2], d[3]) << 16);
-    r.y = cvt_e4m3x2(d[4], d[5]) | (cvt_e4m3x2(d[6], d[7]) << 16);
-    return r;
+// ---------------------------------------------------------------------------
+// E4M3 code of the IEEE fp32 quotient x / s, without a division per element.
+//
+// The code must equal E(RN32(x / s)) where E is the (monotone, saturating,
+// round-to-nearest-even) E4M3 conversion.  With r = RN32(1 / s) (the
+// correctly rounded reciprocal, __frcp_rn) and q = RN32(x * r):
+//   |q - x/s| <= 2^-23 |x/s| (two roundings of 2^-24 each), and
+//   |RN32(x/s) - x/s| <= 2^-24 |x/s|,
+// so RN32(x/s) lies between q(1 - 2^-20) and q(1 + 2^-20).  E is monotone,
+// hence when E(q(1 - 2^-20)) == E(q(1 + 2^-20)) that common code is
+// E(RN32(x/s)).  Otherwise (x/s within ~2^-20 of an E4M3 rounding midpoint,
+// a fraction ~2e-5 of inputs) the pair is recomputed with IEEE division.
+// The bounds need s and 1/s to be normal fp32 numbers: tiles whose scale is
+// outside [2^-125, 2^125] use IEEE division throughout.  Signs, zeros, NaN
+// and the saturation at 448 carry through both ends unchanged.
+// ---------------------------------------------------------------------------
+constexpr float kBracketUp = 1.0f + 0x1p-20f;
+constexpr float kBracketDown = 1.0f - 0x1p-20f;
+
+__device__ __forceinline__ bool reciprocal_path_ok(float s) {
+    return s >= 0x1p-125f && s <= 0x1p125f;
 }
+
+__device__ __forceinline__ uint32_t encode_pair(float x0, float x1, float s, float r) {
+    const float q0 = x0 * r;
+    const float q1 = x1 * r;
+    const uint32_t hi = cvt_e4m3x2(q0 * kBracketUp, q1 * kBracketUp);
+    const uint32_t lo = cvt_e4m3x2(q0 * kBracketDown, q1 * kBracketDown);
+    if (hi == lo) return hi;
+    return cvt_e4m3x2(__fdiv_rn(x0, s), __fdiv_rn(x1, s));
+}
+
+// 8 values / scale -> 8 E4M3 codes packed little-endian in a uint2.
+// `fast` selects the reciprocal path (reciprocal_path_ok(s)); r = 1/s.
+__device__ __forceinline__ uint2 encode8(const float (&v)[8], float s, float r, bool fast) {
+    uint2 out;
+    if (fast) {
+        out.x = encode_pair(v[0], v[1], s, r) | (encode_pair(v[2], v[3], s, r) << 16);
+        out.y = encode_pair(v[4], v[5], s, r) | (encode_pair(v[6], v[7], s, r) << 16);
+    } else {
+        float d[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) d[i] = __fdiv_rn(v[i], s);
+        out.x = cvt_e4m3x2(d[0], d[1]) | (cvt_e4m3x2(d[2], d[3]) << 16);
+        out.y = cvt_e4m3x2(d[4], d[5]) | (cvt_e4m3x2(d[6], d[7]) << 16);
+    }
+    return out;
+}
+
+// floor(n / d) for 0 <= n < 2^31 and a fixed d >= 1, by multiplication:
+// with l = ceil(log2 d) and m = ceil(2^(31+l) / d), 2^(31+l) <= m d <=
+// 2^(31+l) + 2^l, so floor(n / d) = (n m) >> (31 + l) (Granlund and
+// Montgomery, "Division by invariant integers using multiplication", 1994,
+// round-up method).  m <= 2^32 keeps n m below 2^63.
+struct FastDivU31 {
+    uint64_t m;
+    int shift;
+    __host__ static FastDivU31 make(uint32_t d) {  // d < 2^31
+        int l = 0;
+        while ((static_cast<uint64_t>(1) << l) < d) ++l;
+        FastDivU31 f;
+        const uint64_t num = static_cast<uint64_t>(1) << (31 + l);  // l <= 31
+        f.m = (num + d - 1) / d;
+        f.shift = 31 + l;
+        return f;
+    }
+    __device__ __forceinline__ uint32_t div(uint32_t n) const {
+        return static_cast<uint32_t>((static_cast<uint64_t>(n) * m) >> shift);
+    }
+};
 
 // ---------------------------------------------------------------------------
 // 1x128 activation tiles.  A half-warp owns one tile: lane l of the half
@@ -69,11 +129,13 @@ __device__ __forceinline__ uint2 encode8(const float (&v)[8], float s) {
 constexpr int kActThreads = 256;
 constexpr int kActUnroll = 4;
 
-template <typename T>
+// kSmall: M * nkb < 2^31, tile index -> (row, kb) by FastDivU31; otherwise
+// 64-bit division.
+template <typename T, bool kSmall>
 __global__ void __launch_bounds__(kActThreads)
-    quant_act_1x128_kernel(const T* __restrict__ x, int64_t M, int64_t nkb, int64_t ldx,
-                           uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sa,
-                           int64_t sa_sm, int64_t sa_skb) {
+    quant_act_1x128_kernel(const T* __restrict__ x, int64_t M, int64_t nkb, FastDivU31 fd,
+                           int64_t ldx, uint8_t* __restrict__ q, int64_t ldq,
+                           float* __restrict__ sa, int64_t sa_sm, int64_t sa_skb) {
     const int hl = threadIdx.x & 15;          // lane within the half-warp
     const int hw = threadIdx.x >> 4;          // half-warp within the block (0..15)
     const int64_t total = M * nkb;
@@ -86,8 +148,14 @@ __global__ void __launch_bounds__(kActThreads)
 #pragma unroll
         for (int u = 0; u < kActUnroll; ++u) {
             const int64_t t = base + u * 16 + hw;
-            row[u] = t / nkb;
-            kb[u] = t - row[u] * nkb;
+            if (kSmall) {
+                const uint32_t t32 = t < total ? static_cast<uint32_t>(t) : 0u;
+                row[u] = fd.div(t32);
+                kb[u] = static_cast<int64_t>(t32) - row[u] * nkb;
+            } else {
+                row[u] = t / nkb;
+                kb[u] = t - row[u] * nkb;
+            }
             if (t < total) {
                 InVec<T>::load(x + row[u] * ldx + kb[u] * 128 + hl * 8, v[u]);
             } else {
@@ -104,9 +172,10 @@ __global__ void __launch_bounds__(kActThreads)
             for (int off = 8; off > 0; off >>= 1)
                 amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
             const float s = scale_from_amax(amax);
+            const float r = __frcp_rn(s);
             const int64_t t = base + u * 16 + hw;
             if (t < total) {
-                const uint2 codes = encode8(v[u], s);
+                const uint2 codes = encode8(v[u], s, r, reciprocal_path_ok(s));
                 __stcs(reinterpret_cast<uint2*>(q + row[u] * ldq + kb[u] * 128 + hl * 8), codes);
                 if (hl == 0) sa[row[u] * sa_sm + kb[u] * sa_skb] = s;
             }
@@ -161,11 +230,13 @@ __global__ void __launch_bounds__(kWThreads)
 #pragma unroll
         for (int i = 1; i < kWThreads / 32; ++i) amax = fmaxf(amax, red[i]);
         const float s = scale_from_amax(amax);
+        const float rcp = __frcp_rn(s);
+        const bool fast = reciprocal_path_ok(s);
         if (tid == 0) sb[kb * sb_skb + nb * sb_snb] = s;
 
         uint2 codes[8];
 #pragma unroll
-        for (int r = 0; r < 8; ++r) codes[r] = encode8(v[r], s);
+        for (int r = 0; r < 8; ++r) codes[r] = encode8(v[r], s, rcp, fast);
 
         if (!transpose_out) {
             uint8_t* dst = q + (kb * 128) * ldq + nb * 128 + c * 8;

@@ -142,6 +142,35 @@ __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// tcgen05.wait::ld that also "redefines" the 32 destination registers of the
+// preceding tcgen05.ld, so that no use of them can be scheduled before the
+// wait (the load writes them asynchronously).
+__device__ __forceinline__ void tmem_wait_ld_dep(uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.wait::ld.sync.aligned;"
+        : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+          "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
+          "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]),
+          "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
+          "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]),
+          "+r"(r[31])
+        :
+        : "memory");
+}
+
+// Packed FP32 FMA on sm_100: (d0, d1) = s * (b0, b1) + (d0, d1), each lane
+// rounded to nearest even like fmaf.
+__device__ __forceinline__ void ffma2_scalar(float& d0, float& d1, float s, float b0, float b1) {
+    asm("{\n\t.reg .b64 ta, tb, td;\n\t"
+        "mov.b64 ta, {%2, %2};\n\t"
+        "mov.b64 tb, {%3, %4};\n\t"
+        "mov.b64 td, {%0, %1};\n\t"
+        "fma.rn.f32x2 td, ta, tb, td;\n\t"
+        "mov.b64 {%0, %1}, td;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(s), "f"(b0), "f"(b1));
+}
+
 // Shared-memory matrix descriptor (tcgen05 format) for a K-major operand
 // tile laid out by TMA with 128-byte swizzling: rows of 128 bytes, groups of
 // 8 rows 1024 bytes apart.  The tile base must be 1024-byte aligned.

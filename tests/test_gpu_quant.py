@@ -82,6 +82,39 @@ def test_cvt_rounding_matches_oracle_encoder(cuda_lib, orc):
     assert_codes_equal(np_u8(q), orc.e4m3_encode(tiles))
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_quotients_at_rounding_midpoints(cuda_lib, orc, dtype):
+    """Tiles with non-power-of-two scales whose elements are (a few ulps
+    around) E4M3 midpoints times the scale: x / s lands within a few fp32
+    ulps of a rounding boundary, where a reciprocal-based quotient could
+    round differently from the IEEE quotient."""
+    rng = np.random.default_rng(7)
+    dec = orc.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+    mids = (dec[:-1] + dec[1:]) / 2
+    rows = 4096
+    tiles = np.empty((rows, 128), dtype=np.float32)
+    amax = (rng.uniform(0.5, 2.0, rows) * np.exp2(rng.integers(-30, 30, rows))).astype(np.float32)
+    if dtype == torch.bfloat16:    # amax itself must survive the bf16 rounding
+        amax = torch.from_numpy(amax).bfloat16().float().numpy()
+    s = (amax / np.float32(448.0)).astype(np.float32)
+    m = rng.choice(mids, size=(rows, 127)) * rng.choice([-1.0, 1.0], size=(rows, 127))
+    x = (m * s[:, None].astype(np.float64)).astype(np.float32)
+    jitter = rng.integers(-3, 4, size=x.shape).astype(np.int32)
+    x = (x.view(np.int32) + jitter).view(np.float32)
+    tiles[:, 0] = amax
+    tiles[:, 1:] = np.clip(x, -amax[:, None], amax[:, None])
+    xt = torch.from_numpy(tiles).to(dtype)
+    q, sa = cuda_lib.fp8_quantize_act_1x128(xt.cuda())
+    qo, sao = orc.quantize_act_1x128(to_oracle(xt))
+    assert_codes_equal(np_u8(q), qo)
+    assert_scales_equal(sa.cpu().numpy(), sao)
+    w = xt[:1024].reshape(128, 1024)                # same values through the weight kernel
+    qw, sw = cuda_lib.fp8_quantize_weight_128x128(w.cuda(), transpose_out=True)
+    qwo, swo = orc.quantize_weight_128x128(to_oracle(w), transpose_out=True)
+    assert_codes_equal(np_u8(qw), qwo)
+    assert_scales_equal(sw.cpu().numpy(), swo)
+
+
 def test_act_quant_nan_element_smoke(cuda_lib, orc):
     """Out of contract: a NaN element is skipped by amax and encodes to NaN."""
     x = torch.randn(2, 256)
@@ -110,7 +143,7 @@ def test_weight_quant_bit_exact(cuda_lib, orc, K, N, dtype, transpose):
 def test_weight_quant_zero_and_strided(cuda_lib, orc):
     K, N = 256, 384
     big = synth.normal((K, 512), 0.02, 5, "cpu", torch.float32)
-    big[:128, :128] = 0.0
+    big[:128, 64:192] = 0.0                        # block (0, 0) of the slice below
     w = big[:, 64:64 + N].cuda()
     sbT = torch.zeros((N // 128, K // 128), device="cuda")
     for transpose in (False, True):
