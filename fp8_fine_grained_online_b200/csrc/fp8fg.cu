@@ -13,6 +13,7 @@
 
 #include "../../include/fp8fg.h"
 #include "gemm_kernels.cuh"
+#include "gemm_pair_kernels.cuh"
 #include "quant_kernels.cuh"
 
 namespace fp8fg {
@@ -23,6 +24,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
     std::atomic<int> state{0};  // 0 unknown, 1 ok, 2 unsupported
     int num_sms = 0;
+    int max_pairs = 0;          // co-resident 2-CTA clusters of the pair GEMM
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -62,6 +64,38 @@ fp8_status_t current_device(int* dev_out, int* sms_out) {
                         return FP8_ERR_CUDA;
                     }
                 }
+                const void* pair_kernels[] = {
+                    reinterpret_cast<const void*>(&blockscaled_gemm_pair_kernel<false>),
+                    reinterpret_cast<const void*>(&blockscaled_gemm_pair_kernel<true>)};
+                for (const void* k : pair_kernels) {
+                    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kGemmPairSmemBytes)) != cudaSuccess) {
+                        cudaGetLastError();
+                        return FP8_ERR_CUDA;
+                    }
+                }
+                // CTA pairs that can be resident at once (a cluster must fit in
+                // one GPC): the persistent grid must not exceed it, or the
+                // surplus pairs would run as a second wave.
+                cudaLaunchConfig_t cfg = {};
+                cfg.gridDim = dim3(2, 1, 1);
+                cfg.blockDim = dim3(kGemmThreads, 1, 1);
+                cfg.dynamicSmemBytes = kGemmPairSmemBytes;
+                cudaLaunchAttribute attr[1];
+                attr[0].id = cudaLaunchAttributeClusterDimension;
+                attr[0].val.clusterDim.x = 2;
+                attr[0].val.clusterDim.y = 1;
+                attr[0].val.clusterDim.z = 1;
+                cfg.attrs = attr;
+                cfg.numAttrs = 1;
+                int clusters = 0;
+                if (cudaOccupancyMaxActiveClusters(&clusters, blockscaled_gemm_pair_kernel<true>,
+                                                   &cfg) != cudaSuccess ||
+                    clusters < 1) {
+                    cudaGetLastError();
+                    return FP8_ERR_CUDA;
+                }
+                d.max_pairs = clusters;
             }
             d.num_sms = sms;
             st = ok ? 1 : 2;
@@ -184,7 +218,8 @@ fp8_status_t fp8_quantize_act_1x128(const void* x, fp8_in_t x_type, int64_t M, i
 
     const int64_t nkb = K / 128;
     const int64_t tiles = M * nkb;
-    const int64_t per_block = 16 * kActUnroll;
+    const int64_t per_block =
+        16 * (x_type == FP8_IN_BF16 ? act_unroll<uint16_t>() : act_unroll<float>());
     const int64_t grid = grid_for((tiles + per_block - 1) / per_block, sms, 8);
     const bool small = tiles + per_block < (static_cast<int64_t>(1) << 31);
     const FastDivU31 fd = FastDivU31::make(small ? static_cast<uint32_t>(nkb) : 1u);
@@ -269,7 +304,8 @@ fp8_status_t fp8_blockscaled_gemm(const uint8_t* a, int64_t lda, const float* sa
     fp8_status_t st = check_gemm_common(a, lda, sa, sa_stride_m, sa_stride_kb, b, ldb, sb,
                                         sb_stride_kb, sb_stride_nb, c, c_type, ldc, N, K);
     if (st != FP8_OK) return st;
-    const int64_t num_mt = (M + kBM - 1) / kBM, num_nt = (N + kBN - 1) / kBN;
+    // 256 x 256 tiles, one per CTA pair (two SMs).
+    const int64_t num_mt = (M + kPairBM - 1) / kPairBM, num_nt = (N + kBN - 1) / kBN;
     if (num_mt * num_nt > INT32_MAX || M > INT32_MAX) return FP8_ERR_SHAPE;
     int dev, sms;
     st = current_device(&dev, &sms);
@@ -277,8 +313,8 @@ fp8_status_t fp8_blockscaled_gemm(const uint8_t* a, int64_t lda, const float* sa
 
     CUtensorMap tmA, tmB;
     const uint64_t kcols = static_cast<uint64_t>(K);
-    if (!make_operand_map(&tmA, a, static_cast<uint64_t>(M), kcols, static_cast<uint64_t>(lda), kBM) ||
-        !make_operand_map(&tmB, b, static_cast<uint64_t>(N), kcols, static_cast<uint64_t>(ldb), kBN))
+    if (!make_operand_map(&tmA, a, static_cast<uint64_t>(M), kcols, static_cast<uint64_t>(lda), 128) ||
+        !make_operand_map(&tmB, b, static_cast<uint64_t>(N), kcols, static_cast<uint64_t>(ldb), 128))
         return FP8_ERR_CUDA;
 
     GemmParams p{};
@@ -288,15 +324,31 @@ fp8_status_t fp8_blockscaled_gemm(const uint8_t* a, int64_t lda, const float* sa
     p.nkb = static_cast<int>(K / 128);
     p.num_mt = static_cast<int>(num_mt);
     p.num_nt = static_cast<int>(num_nt);
-    p.band_m = 16;
+    p.band_m = 8;     // 2048-row bands: a wave of pairs shares A rows and B columns in L2
     p.offsets = nullptr; p.G = 1;
-    const int64_t grid = grid_for(num_mt * num_nt, sms, 1);
+    const int64_t pairs = grid_for(num_mt * num_nt, g_dev[dev].max_pairs, 1);
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = kGemmPairSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
     if (c_type == FP8_OUT_BF16)
-        blockscaled_gemm_kernel<false, true>
-            <<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, stream>>>(tmA, tmB, p);
+        e = cudaLaunchKernelEx(&cfg, blockscaled_gemm_pair_kernel<true>, tmA, tmB, p);
     else
-        blockscaled_gemm_kernel<false, false>
-            <<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, stream>>>(tmA, tmB, p);
+        e = cudaLaunchKernelEx(&cfg, blockscaled_gemm_pair_kernel<false>, tmA, tmB, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return FP8_ERR_CUDA;
+    }
     return launch_status();
 }
 

@@ -52,7 +52,8 @@ constexpr int kGemmThreads = 384;
 constexpr int kEpiWarps = 8;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr int kSchedWarp = 10;
+constexpr int kMmaWarp2 = 10;   // second MMA issuer of the CTA-pair kernel
+constexpr int kSchedWarp = 10;  // grouped kernel: builds the tile table
 constexpr int kCtrlRegs = 40;
 constexpr int kEpiRegs = 232;
 static_assert(128 * kCtrlRegs + 256 * kEpiRegs <= kGemmThreads * 168, "register split");
@@ -118,15 +119,23 @@ struct TileCoord {
 
 // Wait for phase `parity` of `bar` to complete; false if this CTA aborted or
 // the wait ran past kWaitLimitNs (which aborts the CTA).
+// The limit is counted in SM clock cycles (clock64 is a cheap local
+// counter; the device-wide %globaltimer is slow to read and would delay the
+// reaction to a completed barrier).  2^31 cycles is about one second at the
+// B200's 1.9 GHz and a few seconds at its lowest clocks.
+constexpr long long kWaitLimitCycles = 1ll << 31;
+constexpr int kPollsPerClockCheck = 64;
+
 __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity,
                                              volatile int* abort_flag) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
+    const long long t0 = clock64();
     while (true) {
-        if (mbar_try_wait(a, parity)) return true;
+        for (int i = 0; i < kPollsPerClockCheck; ++i)
+            if (mbar_try_wait(a, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (clock64() - t0 > kWaitLimitCycles) {
             *abort_flag = 1;
             record_device_error(kDevErrTimeout);
             return false;
@@ -134,20 +143,24 @@ __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity,
     }
 }
 
-// Same, ignoring the abort flag: used on the abort path to drain copies
-// and MMAs this thread issued, so that no async write outlives the CTA.
+// Same, ignoring the abort flag: used to drain copies, MMAs and arrivals
+// this CTA is owed, so that no async write outlives the CTA.
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     const uint32_t a = smem_u32(bar);
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(a, parity)) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    const long long t0 = clock64();
+    while (true) {
+        for (int i = 0; i < kPollsPerClockCheck; ++i)
+            if (mbar_try_wait(a, parity)) return;
+        if (clock64() - t0 > kWaitLimitCycles) {
             record_device_error(kDevErrTimeout);
             return;
         }
     }
 }
 
-template <bool kGrouped>
+// Tile t of the persistent schedule.  Dense tiles are kTileM rows high;
+// grouped tiles are kBM rows of one group.
+template <bool kGrouped, int kTileM = kBM>
 __device__ __forceinline__ TileCoord decode_tile(int t, const GemmParams& p,
                                                  const GemmSmemTail* tail) {
     TileCoord tc;
@@ -161,7 +174,7 @@ __device__ __forceinline__ TileCoord decode_tile(int t, const GemmParams& p,
         const int bm = min(p.band_m, p.num_mt - bm0);
         const int nt = within / bm;
         const int mt = bm0 + (within - nt * bm);
-        tc.m0 = static_cast<int64_t>(mt) * kBM;
+        tc.m0 = static_cast<int64_t>(mt) * kTileM;
         tc.row_end = p.M;
         tc.n0 = static_cast<int64_t>(nt) * kBN;
         tc.g = 0;
@@ -193,6 +206,97 @@ __device__ __forceinline__ void promote32(float (&acc)[128], const uint32_t (&pa
     for (int i = 0; i < 32; i += 2)
         ffma2_scalar(acc[kOff + i], acc[kOff + i + 1], s, __uint_as_float(part[i]),
                      __uint_as_float(part[i + 1]));
+}
+
+// One tile of the epilogue, for one thread: promotes every 128-wide K chunk
+// of its row slice (128 columns of the 256-wide tile) from TMEM into FP32
+// registers, acc += sa[row, kb] * sb[kb, nb] * P_kb, then converts and stores
+// the row slice.  `release(buf)` (called by lane 0 after the warp has read
+// its slice of a chunk) hands TMEM buffer `buf` back to the MMA issuer.
+// Returns false if a wait was abandoned because the CTA is aborting.
+template <bool kOutBf16, typename Release>
+__device__ __forceinline__ bool epilogue_tile(const GemmParams& p, uint64_t* tfull,
+                                              volatile int* abort_flag, uint32_t tmem_base,
+                                              uint32_t t_lane, int h, int lane, int64_t row,
+                                              bool row_ok, int64_t col0, bool col_ok, int g,
+                                              uint32_t& chunk, Release release) {
+    const int nkb = p.nkb;
+    const float* sa_row = p.sa + (row_ok ? row : 0) * p.sa_sm;
+    const float* sb_col = p.sb + g * p.sb_sg + (col_ok ? col0 / 128 : 0) * p.sb_snb;
+
+    float acc[128];
+#pragma unroll
+    for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+    float sa_next = (row_ok && nkb > 0) ? __ldg(sa_row) : 0.0f;
+    float sb_next = (col_ok && nkb > 0) ? __ldg(sb_col) : 0.0f;
+
+    // Scales two chunks ahead (the loads are L2 round trips).
+    float sa1 = (row_ok && nkb > 1) ? __ldg(sa_row + p.sa_skb) : 0.0f;
+    float sb1 = (col_ok && nkb > 1) ? __ldg(sb_col + p.sb_skb) : 0.0f;
+
+    // Per chunk: two round trips of 64 columns through 64 staging registers;
+    // the second pair of loads is issued while the first is promoted, and the
+    // TMEM buffer is handed back to the MMA issuer as soon as the last load
+    // has landed, before the second half is promoted.
+    uint32_t pa[32], pb[32];
+    for (int kb = 0; kb < nkb; ++kb) {
+        const float scale = sa_next * sb_next;
+        float sa2 = 0.0f, sb2 = 0.0f;
+        if (kb + 2 < nkb) {
+            sa2 = row_ok ? __ldg(sa_row + (kb + 2) * p.sa_skb) : 0.0f;
+            sb2 = col_ok ? __ldg(sb_col + (kb + 2) * p.sb_skb) : 0.0f;
+        }
+        sa_next = sa1;
+        sb_next = sb1;
+        sa1 = sa2;
+        sb1 = sb2;
+
+        const uint32_t buf = chunk & 1u;
+        if (!bounded_wait(&tfull[buf], (chunk >> 1) & 1u, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + t_lane + buf * kBN + h * 128;
+        tmem_ld_32x32b_x32(taddr, pa);
+        tmem_ld_32x32b_x32(taddr + 32, pb);
+        tmem_wait_ld_dep(pa);
+        tmem_wait_ld_dep(pb);
+        promote32<0>(acc, pa, scale);
+        tmem_ld_32x32b_x32(taddr + 64, pa);
+        promote32<32>(acc, pb, scale);
+        tmem_ld_32x32b_x32(taddr + 96, pb);
+        tmem_wait_ld_dep(pa);
+        tmem_wait_ld_dep(pb);
+        // This warp's slice of the chunk is in registers: hand the TMEM
+        // buffer back to the MMA issuer.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) release(buf);
+        ++chunk;
+        promote32<64>(acc, pa, scale);
+        promote32<96>(acc, pb, scale);
+    }
+    if (row_ok && col_ok) {
+        if (kOutBf16) {
+            __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.c) + row * p.ldc + col0;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const __nv_bfloat162 b2 =
+                        __floats2bfloat162_rn(acc[j * 8 + 2 * e], acc[j * 8 + 2 * e + 1]);
+                    w[e] = *reinterpret_cast<const uint32_t*>(&b2);
+                }
+                reinterpret_cast<uint4*>(out)[j] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        } else {
+            float* out = reinterpret_cast<float*>(p.c) + row * p.ldc + col0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                reinterpret_cast<float4*>(out)[j] =
+                    make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
+        }
+    }
+    return true;
 }
 
 template <bool kGrouped, bool kOutBf16>
@@ -316,12 +420,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 for (int kb = 0; kb < nkb; ++kb) {
                     const uint32_t buf = chunk & 1u;
                     const uint32_t use = chunk >> 1;
-                    if (!bounded_wait(&tail->tempty[buf], (use & 1u) ^ 1u, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    if (!bounded_wait(&tail->full[stage], phase, abort_flag)) {
+                    // Operands first (usually long ready), then the TMEM
+                    // buffer: the epilogue's release is the critical path.
+                    if (!bounded_wait(&tail->full[stage], phase, abort_flag) ||
+                        !bounded_wait(&tail->tempty[buf], (use & 1u) ^ 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -361,82 +463,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const bool row_ok = row < tc.row_end;
             const int64_t col0 = tc.n0 + h * 128;
             const bool col_ok = col0 < p.N;
-            const float* sa_row = p.sa + (row_ok ? row : 0) * p.sa_sm;
-            const float* sb_col = p.sb + tc.g * p.sb_sg + (col_ok ? col0 / 128 : 0) * p.sb_snb;
-
-            float acc[128];
-#pragma unroll
-            for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
-            float sa_next = (row_ok && nkb > 0) ? __ldg(sa_row) : 0.0f;
-            float sb_next = (col_ok && nkb > 0) ? __ldg(sb_col) : 0.0f;
-
-            // Software pipeline over 32-column batches of this warp's 128-column
-            // slice: the TMEM load of the next batch (also across chunk
-            // boundaries) is in flight while the current one is promoted.
-            uint32_t pa[32], pb[32];
-            if (nkb > 0) {
-                if (!bounded_wait(&tail->tfull[chunk & 1u], (chunk >> 1) & 1u, abort_flag)) break;
-                tc_fence_after();
-                tmem_ld_32x32b_x32(tmem_base + t_lane + (chunk & 1u) * kBN + h * 128, pa);
-            }
-            for (int kb = 0; kb < nkb; ++kb) {
-                const float scale = sa_next * sb_next;
-                if (kb + 1 < nkb) {
-                    sa_next = row_ok ? __ldg(sa_row + (kb + 1) * p.sa_skb) : 0.0f;
-                    sb_next = col_ok ? __ldg(sb_col + (kb + 1) * p.sb_skb) : 0.0f;
-                }
-                const uint32_t buf = chunk & 1u;
-                const uint32_t taddr = tmem_base + t_lane + buf * kBN + h * 128;
-                tmem_wait_ld_dep(pa);
-                tmem_ld_32x32b_x32(taddr + 32, pb);
-                promote32<0>(acc, pa, scale);
-                tmem_wait_ld_dep(pb);
-                tmem_ld_32x32b_x32(taddr + 64, pa);
-                promote32<32>(acc, pb, scale);
-                tmem_wait_ld_dep(pa);
-                tmem_ld_32x32b_x32(taddr + 96, pb);
-                promote32<64>(acc, pa, scale);
-                tmem_wait_ld_dep(pb);
-                // This warp's slice of the chunk is in registers: hand the TMEM
-                // buffer back to the MMA warp.
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&tail->tempty[buf]);
-                ++chunk;
-                if (kb + 1 < nkb) {
-                    if (!bounded_wait(&tail->tfull[chunk & 1u], (chunk >> 1) & 1u, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    tmem_ld_32x32b_x32(tmem_base + t_lane + (chunk & 1u) * kBN + h * 128, pa);
-                }
-                promote32<96>(acc, pb, scale);
-            }
-            if (!ok) break;
-            if (row_ok && col_ok) {
-                if (kOutBf16) {
-                    __nv_bfloat16* out =
-                        reinterpret_cast<__nv_bfloat16*>(p.c) + row * p.ldc + col0;
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const __nv_bfloat162 b2 =
-                                __floats2bfloat162_rn(acc[j * 8 + 2 * e], acc[j * 8 + 2 * e + 1]);
-                            w[e] = *reinterpret_cast<const uint32_t*>(&b2);
-                        }
-                        reinterpret_cast<uint4*>(out)[j] = make_uint4(w[0], w[1], w[2], w[3]);
-                    }
-                } else {
-                    float* out = reinterpret_cast<float*>(p.c) + row * p.ldc + col0;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        reinterpret_cast<float4*>(out)[j] =
-                            make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
-                }
-            }
+            ok = epilogue_tile<kOutBf16>(p, tail->tfull, abort_flag, tmem_base, t_lane, h, lane, row,
+                                         row_ok, col0, col_ok, tc.g, chunk,
+                                         [&](uint32_t buf) { mbar_arrive(&tail->tempty[buf]); });
         }
     }
 

@@ -2,7 +2,8 @@
 //
 // Both kernels compute, per tile / block, scale = amax / 448 (IEEE fp32
 // division, 1 when zero) and code = E4M3_RNE_satfinite(x / scale) with one
-// IEEE fp32 division per element (codingmall.com "Kan du förklara rollen
+// IEEE fp32 division per element, evaluated as described at encode_pair
+// (codingmall.com "Kan du förklara rollen
 // för FP8 precision i träningsprocessen för DeepSeek-V3": "Finkornig
 // kvantisering", "Online-kvantisering"; holysheep.ai "FP8 混精度训练
 // DeepSeek 671B" (zh), 2.2).  They are HBM-bound: each input element is
@@ -18,14 +19,20 @@ namespace fp8fg {
 
 constexpr float kE4M3Max = 448.0f;
 
+// Eight consecutive input elements held as raw 16-byte loads, so that the
+// next tile's loads can be issued before the current tile is converted.
 template <typename T>
-struct InVec;  // 8 consecutive input elements, loaded with 16-byte accesses
+struct Raw8;
 
 template <>
-struct InVec<uint16_t> {  // bf16 bit patterns
-    static __device__ __forceinline__ void load(const uint16_t* p, float (&v)[8]) {
-        const uint4 w = __ldcs(reinterpret_cast<const uint4*>(p));
-        const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+struct Raw8<uint16_t> {  // bf16 bit patterns
+    uint4 a;
+    __device__ __forceinline__ void load(const uint16_t* p) {
+        a = __ldcs(reinterpret_cast<const uint4*>(p));
+    }
+    __device__ __forceinline__ void zero() { a = make_uint4(0u, 0u, 0u, 0u); }
+    __device__ __forceinline__ void to_float(float (&v)[8]) const {
+        const uint32_t u[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             v[2 * i] = __uint_as_float(u[i] << 16);           // exact bf16 -> fp32
@@ -35,10 +42,14 @@ struct InVec<uint16_t> {  // bf16 bit patterns
 };
 
 template <>
-struct InVec<float> {
-    static __device__ __forceinline__ void load(const float* p, float (&v)[8]) {
-        const float4 a = __ldcs(reinterpret_cast<const float4*>(p));
-        const float4 b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+struct Raw8<float> {
+    float4 a, b;
+    __device__ __forceinline__ void load(const float* p) {
+        a = __ldcs(reinterpret_cast<const float4*>(p));
+        b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+    }
+    __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ void to_float(float (&v)[8]) const {
         v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
         v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
     }
@@ -124,50 +135,57 @@ struct FastDivU31 {
 // 1x128 activation tiles.  A half-warp owns one tile: lane l of the half
 // loads elements [8l, 8l+8) of it, the tile amax is a 16-lane shuffle
 // reduction, and each lane stores 8 codes.  A block of 256 threads handles
-// 16 * kActUnroll consecutive tiles per step, issuing all loads first.
+// 16 * kActUnroll consecutive tiles per step; the raw loads of the block's
+// next step are issued before the current step is converted, so every lane
+// keeps up to 2 * kActUnroll 16-byte loads in flight.
 // ---------------------------------------------------------------------------
 constexpr int kActThreads = 256;
-constexpr int kActUnroll = 4;
+// Tiles per half-warp per step: 4 for bf16 input, 2 for fp32 (same bytes).
+template <typename T>
+__host__ __device__ constexpr int act_unroll() { return sizeof(T) == 2 ? 4 : 2; }
 
-// kSmall: M * nkb < 2^31, tile index -> (row, kb) by FastDivU31; otherwise
-// 64-bit division.
+// kSmall: M * nkb + step < 2^31, tile index -> (row, kb) by FastDivU31;
+// otherwise 64-bit division.
 template <typename T, bool kSmall>
-__global__ void __launch_bounds__(kActThreads)
+__global__ void __launch_bounds__(kActThreads, 3)
     quant_act_1x128_kernel(const T* __restrict__ x, int64_t M, int64_t nkb, FastDivU31 fd,
                            int64_t ldx, uint8_t* __restrict__ q, int64_t ldq,
                            float* __restrict__ sa, int64_t sa_sm, int64_t sa_skb) {
     const int hl = threadIdx.x & 15;          // lane within the half-warp
     const int hw = threadIdx.x >> 4;          // half-warp within the block (0..15)
+    constexpr int kActUnroll = act_unroll<T>();
     const int64_t total = M * nkb;
     const int64_t step = static_cast<int64_t>(gridDim.x) * (16 * kActUnroll);
 
-    for (int64_t base = static_cast<int64_t>(blockIdx.x) * (16 * kActUnroll); base < total;
-         base += step) {
-        float v[kActUnroll][8];
-        int64_t row[kActUnroll], kb[kActUnroll];
+    auto row_of = [&](int64_t t) -> int64_t {
+        if (kSmall) return static_cast<int64_t>(fd.div(static_cast<uint32_t>(t)));
+        return t / nkb;
+    };
+    auto load_step = [&](int64_t base, Raw8<T> (&raw)[kActUnroll]) {
 #pragma unroll
         for (int u = 0; u < kActUnroll; ++u) {
             const int64_t t = base + u * 16 + hw;
-            if (kSmall) {
-                const uint32_t t32 = t < total ? static_cast<uint32_t>(t) : 0u;
-                row[u] = fd.div(t32);
-                kb[u] = static_cast<int64_t>(t32) - row[u] * nkb;
-            } else {
-                row[u] = t / nkb;
-                kb[u] = t - row[u] * nkb;
-            }
             if (t < total) {
-                InVec<T>::load(x + row[u] * ldx + kb[u] * 128 + hl * 8, v[u]);
+                const int64_t row = row_of(t);
+                raw[u].load(x + row * ldx + (t - row * nkb) * 128 + hl * 8);
             } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) v[u][i] = 0.0f;
+                raw[u].zero();
             }
         }
+    };
+
+    Raw8<T> cur[kActUnroll], nxt[kActUnroll];
+    int64_t base = static_cast<int64_t>(blockIdx.x) * (16 * kActUnroll);
+    load_step(base, cur);
+    for (; base < total; base += step) {
+        load_step(base + step, nxt);
 #pragma unroll
         for (int u = 0; u < kActUnroll; ++u) {
+            float v[8];
+            cur[u].to_float(v);
             float amax = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[u][i]));  // NaN skipped
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));  // NaN skipped
 #pragma unroll
             for (int off = 8; off > 0; off >>= 1)
                 amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
@@ -175,11 +193,15 @@ __global__ void __launch_bounds__(kActThreads)
             const float r = __frcp_rn(s);
             const int64_t t = base + u * 16 + hw;
             if (t < total) {
-                const uint2 codes = encode8(v[u], s, r, reciprocal_path_ok(s));
-                __stcs(reinterpret_cast<uint2*>(q + row[u] * ldq + kb[u] * 128 + hl * 8), codes);
-                if (hl == 0) sa[row[u] * sa_sm + kb[u] * sa_skb] = s;
+                const int64_t row = row_of(t);
+                const int64_t kb = t - row * nkb;
+                const uint2 codes = encode8(v, s, r, reciprocal_path_ok(s));
+                __stcs(reinterpret_cast<uint2*>(q + row * ldq + kb * 128 + hl * 8), codes);
+                if (hl == 0) sa[row * sa_sm + kb * sa_skb] = s;
             }
         }
+#pragma unroll
+        for (int u = 0; u < kActUnroll; ++u) cur[u] = nxt[u];
     }
 }
 
@@ -193,7 +215,7 @@ __global__ void __launch_bounds__(kActThreads)
 constexpr int kWThreads = 256;
 
 template <typename T>
-__global__ void __launch_bounds__(kWThreads)
+__global__ void __launch_bounds__(kWThreads, sizeof(T) == 2 ? 2 : 1)
     quant_weight_128x128_kernel(const T* __restrict__ w, int64_t nkb, int64_t nnb, int64_t ldw,
                                 uint8_t* __restrict__ q, int transpose_out, int64_t ldq,
                                 float* __restrict__ sb, int64_t sb_skb, int64_t sb_snb) {
@@ -204,23 +226,32 @@ __global__ void __launch_bounds__(kWThreads)
     const int c = tid & 15;
     const int kq = tid >> 4;
     const int64_t nblocks = nkb * nnb;
-
-    for (int64_t blk = blockIdx.x; blk < nblocks; blk += gridDim.x) {
+    // Row of slot r (0..7) of this thread within a 128-row block.
+    auto row_in_block = [&](int r) { return (r >> 2) * 64 + kq * 4 + (r & 3); };
+    auto load_block = [&](int64_t blk, Raw8<T> (&raw)[8]) {
         const int64_t kb = blk / nnb;
         const int64_t nb = blk - kb * nnb;
         const T* src = w + (kb * 128) * ldw + nb * 128 + c * 8;
-
-        float v[8][8];  // [row slot][column]
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            const int k = (r >> 2) * 64 + kq * 4 + (r & 3);
-            InVec<T>::load(src + k * ldw, v[r]);
-        }
+        for (int r = 0; r < 8; ++r) raw[r].load(src + row_in_block(r) * ldw);
+    };
+
+    Raw8<T> cur[8], nxt[8];
+    int64_t blk = blockIdx.x;
+    if (blk < nblocks) load_block(blk, cur);
+    for (; blk < nblocks; blk += gridDim.x) {
+        const int64_t kb = blk / nnb;
+        const int64_t nb = blk - kb * nnb;
+        if (blk + gridDim.x < nblocks) load_block(blk + gridDim.x, nxt);
+
         float amax = 0.0f;
 #pragma unroll
-        for (int r = 0; r < 8; ++r)
+        for (int r = 0; r < 8; ++r) {
+            float v[8];
+            cur[r].to_float(v);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[r][i]));
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1)
             amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
@@ -236,15 +267,17 @@ __global__ void __launch_bounds__(kWThreads)
 
         uint2 codes[8];
 #pragma unroll
-        for (int r = 0; r < 8; ++r) codes[r] = encode8(v[r], s, rcp, fast);
+        for (int r = 0; r < 8; ++r) {
+            float v[8];
+            cur[r].to_float(v);
+            codes[r] = encode8(v, s, rcp, fast);
+        }
 
         if (!transpose_out) {
             uint8_t* dst = q + (kb * 128) * ldq + nb * 128 + c * 8;
 #pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                const int k = (r >> 2) * 64 + kq * 4 + (r & 3);
-                __stcs(reinterpret_cast<uint2*>(dst + k * ldq), codes[r]);
-            }
+            for (int r = 0; r < 8; ++r)
+                __stcs(reinterpret_cast<uint2*>(dst + row_in_block(r) * ldq), codes[r]);
         } else {
             // Gather, per column n, the 4 codes of rows 4kq..4kq+3 (and the
             // +64 group) into one word: tbuf[n][k/4].
@@ -278,6 +311,8 @@ __global__ void __launch_bounds__(kWThreads)
             }
         }
         __syncthreads();  // red[] and tbuf[] are reused by the next block
+#pragma unroll
+        for (int r = 0; r < 8; ++r) cur[r] = nxt[r];
     }
 }
 
