@@ -15,6 +15,8 @@
 #include "gemm_kernels.cuh"
 #include "gemm_pair_kernels.cuh"
 #include "quant_kernels.cuh"
+#include "quant_stream_kernels.cuh"
+#include "quant_act_kernels.cuh"
 
 namespace fp8fg {
 namespace {
@@ -70,6 +72,25 @@ fp8_status_t current_device(int* dev_out, int* sms_out) {
                 for (const void* k : pair_kernels) {
                     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(kGemmPairSmemBytes)) != cudaSuccess) {
+                        cudaGetLastError();
+                        return FP8_ERR_CUDA;
+                    }
+                }
+                const void* qs_bf16[] = {
+                    reinterpret_cast<const void*>(&quant_stream_kernel<uint16_t, kQuantAct>),
+                    reinterpret_cast<const void*>(&quant_stream_kernel<uint16_t, kQuantWeight>),
+                    reinterpret_cast<const void*>(&quant_stream_kernel<uint16_t, kQuantWeightT>)};
+                const void* qs_f32[] = {
+                    reinterpret_cast<const void*>(&quant_stream_kernel<float, kQuantAct>),
+                    reinterpret_cast<const void*>(&quant_stream_kernel<float, kQuantWeight>),
+                    reinterpret_cast<const void*>(&quant_stream_kernel<float, kQuantWeightT>)};
+                for (int i = 0; i < 3; ++i) {
+                    if (cudaFuncSetAttribute(qs_bf16[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(quant_stream_smem_bytes<uint16_t>())) !=
+                            cudaSuccess ||
+                        cudaFuncSetAttribute(qs_f32[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(quant_stream_smem_bytes<float>())) !=
+                            cudaSuccess) {
                         cudaGetLastError();
                         return FP8_ERR_CUDA;
                     }
@@ -177,6 +198,54 @@ fp8_status_t zero_output(void* c, fp8_out_t ct, int64_t ldc, int64_t rows, int64
     return launch_status();
 }
 
+
+// 2-D input tensor [rows, cols] (bf16 or fp32) with row stride `ld`
+// elements, box 128 x 128, no swizzle, zero fill out of bounds.
+bool make_input_map(CUtensorMap* map, const void* base, fp8_in_t t, uint64_t rows, uint64_t cols,
+                    uint64_t ld) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const int es = elem_size_in(t);
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {ld * static_cast<uint64_t>(es)};
+    cuuint32_t box[2] = {128, 128};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, t == FP8_IN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                     2, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <typename T, int kMode>
+fp8_status_t launch_quant_stream_t(const CUtensorMap& map, const QsParams& p, int sms,
+                                   cudaStream_t stream) {
+    const int64_t boxes = p.nbr * p.nbc;
+    const unsigned grid = static_cast<unsigned>(boxes < sms ? boxes : sms);
+    quant_stream_kernel<T, kMode>
+        <<<grid, kQsThreads, quant_stream_smem_bytes<T>(), stream>>>(map, p);
+    return launch_status();
+}
+
+// One persistent CTA per SM streams the 128x128 boxes of the input.
+fp8_status_t launch_quant_stream(const void* in, fp8_in_t t, int64_t ld, const QsParams& p,
+                                 int mode, int sms, cudaStream_t stream) {
+    CUtensorMap map;
+    if (!make_input_map(&map, in, t, static_cast<uint64_t>(p.rows), static_cast<uint64_t>(p.cols),
+                        static_cast<uint64_t>(ld)))
+        return FP8_ERR_CUDA;
+    if (t == FP8_IN_BF16) {
+        if (mode == kQuantAct) return launch_quant_stream_t<uint16_t, kQuantAct>(map, p, sms, stream);
+        if (mode == kQuantWeight)
+            return launch_quant_stream_t<uint16_t, kQuantWeight>(map, p, sms, stream);
+        return launch_quant_stream_t<uint16_t, kQuantWeightT>(map, p, sms, stream);
+    }
+    if (mode == kQuantAct) return launch_quant_stream_t<float, kQuantAct>(map, p, sms, stream);
+    if (mode == kQuantWeight) return launch_quant_stream_t<float, kQuantWeight>(map, p, sms, stream);
+    return launch_quant_stream_t<float, kQuantWeightT>(map, p, sms, stream);
+}
+
 }  // namespace
 }  // namespace fp8fg
 
@@ -212,16 +281,14 @@ fp8_status_t fp8_quantize_act_1x128(const void* x, fp8_in_t x_type, int64_t M, i
     if (ldx < K || ldq < K || sa_stride_m < 0 || sa_stride_kb < 0) return FP8_ERR_LAYOUT;
     if (!aligned16(x) || (ldx * es) % 16 != 0 || !aligned16(q) || ldq % 16 != 0 || !aligned4(sa))
         return FP8_ERR_ALIGN;
+    if (M > INT32_MAX) return FP8_ERR_SHAPE;
     int dev, sms;
     fp8_status_t st = current_device(&dev, &sms);
     if (st != FP8_OK) return st;
-
     const int64_t nkb = K / 128;
     const int64_t tiles = M * nkb;
-    const int64_t per_block =
-        16 * (x_type == FP8_IN_BF16 ? act_unroll<uint16_t>() : act_unroll<float>());
-    const int64_t grid = grid_for((tiles + per_block - 1) / per_block, sms, 8);
-    const bool small = tiles + per_block < (static_cast<int64_t>(1) << 31);
+    const int64_t grid = grid_for((tiles + kActTilesPerStep - 1) / kActTilesPerStep, sms, 2);
+    const bool small = tiles + grid * kActTilesPerStep < (static_cast<int64_t>(1) << 31);
     const FastDivU31 fd = FastDivU31::make(small ? static_cast<uint32_t>(nkb) : 1u);
     const unsigned g = static_cast<unsigned>(grid);
     if (x_type == FP8_IN_BF16) {
@@ -257,21 +324,17 @@ fp8_status_t fp8_quantize_weight_128x128(const void* w, fp8_in_t w_type, int64_t
         return FP8_ERR_LAYOUT;
     if (!aligned16(w) || (ldw * es) % 16 != 0 || !aligned16(q) || ldq % 16 != 0 || !aligned4(sb))
         return FP8_ERR_ALIGN;
+    if (K > INT32_MAX || N > INT32_MAX) return FP8_ERR_SHAPE;
     int dev, sms;
     fp8_status_t st = current_device(&dev, &sms);
     if (st != FP8_OK) return st;
-
-    const int64_t nkb = K / 128, nnb = N / 128;
-    const int64_t grid = grid_for(nkb * nnb, sms, 8);
-    if (w_type == FP8_IN_BF16)
-        quant_weight_128x128_kernel<uint16_t><<<static_cast<unsigned>(grid), kWThreads, 0, stream>>>(
-            static_cast<const uint16_t*>(w), nkb, nnb, ldw, q, transpose_out ? 1 : 0, ldq, sb,
-            sb_stride_kb, sb_stride_nb);
-    else
-        quant_weight_128x128_kernel<float><<<static_cast<unsigned>(grid), kWThreads, 0, stream>>>(
-            static_cast<const float*>(w), nkb, nnb, ldw, q, transpose_out ? 1 : 0, ldq, sb,
-            sb_stride_kb, sb_stride_nb);
-    return launch_status();
+    QsParams p{};
+    p.rows = K; p.cols = N;
+    p.nbr = K / 128; p.nbc = N / 128;
+    p.q = q; p.ldq = ldq;
+    p.s = sb; p.s_stride_r = sb_stride_kb; p.s_stride_c = sb_stride_nb;
+    return launch_quant_stream(w, w_type, ldw, p, transpose_out ? kQuantWeightT : kQuantWeight,
+                               sms, stream);
 }
 
 static fp8_status_t check_gemm_common(const uint8_t* a, int64_t lda, const float* sa,
