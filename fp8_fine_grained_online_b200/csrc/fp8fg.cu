@@ -77,14 +77,12 @@ fp8_status_t current_device(int* dev_out, int* sms_out) {
                     }
                 }
                 const void* qs_bf16[] = {
-                    reinterpret_cast<const void*>(&quant_stream_kernel<uint16_t, kQuantAct>),
                     reinterpret_cast<const void*>(&quant_stream_kernel<uint16_t, kQuantWeight>),
                     reinterpret_cast<const void*>(&quant_stream_kernel<uint16_t, kQuantWeightT>)};
                 const void* qs_f32[] = {
-                    reinterpret_cast<const void*>(&quant_stream_kernel<float, kQuantAct>),
                     reinterpret_cast<const void*>(&quant_stream_kernel<float, kQuantWeight>),
                     reinterpret_cast<const void*>(&quant_stream_kernel<float, kQuantWeightT>)};
-                for (int i = 0; i < 3; ++i) {
+                for (int i = 0; i < 2; ++i) {
                     if (cudaFuncSetAttribute(qs_bf16[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(quant_stream_smem_bytes<uint16_t>())) !=
                             cudaSuccess ||
@@ -236,12 +234,10 @@ fp8_status_t launch_quant_stream(const void* in, fp8_in_t t, int64_t ld, const Q
                         static_cast<uint64_t>(ld)))
         return FP8_ERR_CUDA;
     if (t == FP8_IN_BF16) {
-        if (mode == kQuantAct) return launch_quant_stream_t<uint16_t, kQuantAct>(map, p, sms, stream);
         if (mode == kQuantWeight)
             return launch_quant_stream_t<uint16_t, kQuantWeight>(map, p, sms, stream);
         return launch_quant_stream_t<uint16_t, kQuantWeightT>(map, p, sms, stream);
     }
-    if (mode == kQuantAct) return launch_quant_stream_t<float, kQuantAct>(map, p, sms, stream);
     if (mode == kQuantWeight) return launch_quant_stream_t<float, kQuantWeight>(map, p, sms, stream);
     return launch_quant_stream_t<float, kQuantWeightT>(map, p, sms, stream);
 }
@@ -287,7 +283,7 @@ fp8_status_t fp8_quantize_act_1x128(const void* x, fp8_in_t x_type, int64_t M, i
     if (st != FP8_OK) return st;
     const int64_t nkb = K / 128;
     const int64_t tiles = M * nkb;
-    const int64_t grid = grid_for((tiles + kActTilesPerStep - 1) / kActTilesPerStep, sms, 2);
+    const int64_t grid = grid_for((tiles + kActTilesPerStep - 1) / kActTilesPerStep, sms, kActMinBlocks);
     const bool small = tiles + grid * kActTilesPerStep < (static_cast<int64_t>(1) << 31);
     const FastDivU31 fd = FastDivU31::make(small ? static_cast<uint32_t>(nkb) : 1u);
     const unsigned g = static_cast<unsigned>(grid);
@@ -387,7 +383,11 @@ fp8_status_t fp8_blockscaled_gemm(const uint8_t* a, int64_t lda, const float* sa
     p.nkb = static_cast<int>(K / 128);
     p.num_mt = static_cast<int>(num_mt);
     p.num_nt = static_cast<int>(num_nt);
-    p.band_m = 8;     // 2048-row bands: a wave of pairs shares A rows and B columns in L2
+    // Bands of m-tiles whose A rows (band_m x 256 rows x K bytes) stay in
+    // L2 (about 40 MB of the 126 MB) while the pairs walk across N: B is
+    // then read from HBM once per band, A once.
+    const int64_t band = (int64_t{40} << 20) / (static_cast<int64_t>(kPairBM) * K);
+    p.band_m = static_cast<int>(band < 1 ? 1 : (band > num_mt ? num_mt : band));
     p.offsets = nullptr; p.G = 1;
     const int64_t pairs = grid_for(num_mt * num_nt, g_dev[dev].max_pairs, 1);
 

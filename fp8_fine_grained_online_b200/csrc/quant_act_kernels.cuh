@@ -6,24 +6,26 @@
 //
 // HBM-bound; straight from registers.  A half-warp owns a tile (lane l of
 // the half holds elements [8l, 8l+8) as one 16-byte load).  A block of 256
-// threads takes 128 consecutive tiles per step: half-warp h gets tiles
-// h, h+16, ..., h+112, so each lane issues 8 independent 16-byte loads
-// before it needs any of them; latency is hidden by those and by occupancy
-// (two blocks, 16 warps per SM).  For its j-th tile the half-warp reduces
-// amax with shuffles, lanes j and j+8 compute the scale and reciprocal once,
-// and the half-warp takes them by shuffle, so no lane divides per element.
+// threads takes kActTilesPerStep consecutive tiles per step: half-warp h
+// gets tiles h, h+16, ..., so each lane issues kActTilesPerLane independent
+// 16-byte loads before it needs any of them; latency is hidden by those and
+// by occupancy (kActMinBlocks blocks per SM).  For its j-th tile the
+// half-warp reduces amax with shuffles, the lanes l = j (mod
+// kActTilesPerLane) compute the scale and reciprocal once, and the
+// half-warp takes them by shuffle, so no lane divides per element.
 #pragma once
 
 #include <cstdint>
 #include <cuda_runtime.h>
 
 #include "quant_kernels.cuh"
-#include "quant_stream_kernels.cuh"   // row_amax8
 
 namespace fp8fg {
 
 constexpr int kActThreads = 256;
-constexpr int kActTilesPerStep = 128;
+constexpr int kActTilesPerLane = 4;                       // tiles a half-warp holds per step
+constexpr int kActMinBlocks = 4;                          // resident blocks per SM
+constexpr int kActTilesPerStep = 16 * kActTilesPerLane;   // 16 half-warps per block
 
 template <typename T>
 __device__ __forceinline__ void load_raw_global(const T* p, Raw8<T>& r);
@@ -48,9 +50,52 @@ __device__ __forceinline__ void zero_raw<float>(Raw8<float>& r) {
     r.a = r.b = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
+// amax[j] = max |x| over tile j of the half-warp (all 16 lanes get it).
+template <typename T, int kJ>
+__device__ __forceinline__ void half_warp_amax(const Raw8<T> (&raw)[kJ], float (&amax)[kJ]);
+
+// bf16: a tile maximum is an exact bf16 value, so two tiles travel in one
+// register and are reduced with packed bf16 maxima.
+template <int kJ>
+__device__ __forceinline__ void half_warp_amax_bf16(const Raw8<uint16_t> (&raw)[kJ],
+                                                    float (&amax)[kJ]) {
+    static_assert(kJ % 2 == 0, "tiles are reduced in pairs");
+#pragma unroll
+    for (int j = 0; j < kJ; j += 2) {
+        const uint32_t a0 = __float_as_uint(raw[j].abs_max()) >> 16;
+        const uint32_t a1 = __float_as_uint(raw[j + 1].abs_max()) & 0xFFFF0000u;
+        uint32_t m = a0 | a1;
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1)
+            m = bf16x2_max(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+        amax[j] = __uint_as_float(m << 16);
+        amax[j + 1] = __uint_as_float(m & 0xFFFF0000u);
+    }
+}
+
+template <int kJ>
+__device__ __forceinline__ void half_warp_amax_f32(const Raw8<float> (&raw)[kJ],
+                                                   float (&amax)[kJ]) {
+#pragma unroll
+    for (int j = 0; j < kJ; ++j) {
+        float a = raw[j].abs_max();
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+        amax[j] = a;
+    }
+}
+
+template <typename T, int kJ>
+__device__ __forceinline__ void half_warp_amax(const Raw8<T> (&raw)[kJ], float (&amax)[kJ]) {
+    if constexpr (sizeof(T) == 2)
+        half_warp_amax_bf16<kJ>(raw, amax);
+    else
+        half_warp_amax_f32<kJ>(raw, amax);
+}
+
 // kSmall: M * nkb + step < 2^31 (tile index -> row by FastDivU31).
 template <typename T, bool kSmall>
-__global__ void __launch_bounds__(kActThreads, 2)
+__global__ void __launch_bounds__(kActThreads, kActMinBlocks)
     quant_act_1x128_kernel(const T* __restrict__ x, int64_t M, int64_t nkb, FastDivU31 fd,
                            int64_t ldx, uint8_t* __restrict__ q, int64_t ldq,
                            float* __restrict__ sa, int64_t sa_sm, int64_t sa_skb) {
@@ -65,9 +110,9 @@ __global__ void __launch_bounds__(kActThreads, 2)
         if (kSmall) return static_cast<int64_t>(fd.div(static_cast<uint32_t>(t)));
         return t / nkb;
     };
-    auto load_step = [&](int64_t base, Raw8<T> (&raw)[8]) {
+    auto load_step = [&](int64_t base, Raw8<T> (&raw)[kActTilesPerLane]) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < kActTilesPerLane; ++j) {
             const int64_t t = base + j * 16 + hw;
             if (t < total) {
                 const int64_t row = row_of(t);
@@ -78,53 +123,69 @@ __global__ void __launch_bounds__(kActThreads, 2)
         }
     };
 
-    Raw8<T> cur[8];
+    Raw8<T> cur[kActTilesPerLane];
     for (int64_t base = static_cast<int64_t>(blockIdx.x) * kActTilesPerStep; base < total;
          base += step) {
         load_step(base, cur);
 
-        float amax[8];
-        row_amax8<T>(cur, amax);
+        float amax[kActTilesPerLane];
+        half_warp_amax<T, kActTilesPerLane>(cur, amax);
         float my_amax = amax[0];
 #pragma unroll
-        for (int j = 1; j < 8; ++j)
-            if ((hl & 7) == j) my_amax = amax[j];
+        for (int j = 1; j < kActTilesPerLane; ++j)
+            if (hl % kActTilesPerLane == j) my_amax = amax[j];
         const float my_s = scale_from_amax(my_amax);
         const float my_r = __frcp_rn(my_s);
-        const float my_ru = my_r * kBracketUp;
-        const float my_rd = my_r * kBracketDown;
 
-        float sj[8];
-        uint32_t bad = 0;
+        // Codes are stored tile by tile.  bf16 input takes the corrected
+        // quotient; fp32 input the bracket, whose ambiguous pairs (bit
+        // 4j + k: pair k of tile j) are then recomputed with IEEE division
+        // and their two bytes overwritten.  Tiles with a scale off the fast
+        // paths go through the same loop, all pairs.
+        float sj[kActTilesPerLane];
+        uint32_t amb = 0;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < kActTilesPerLane; ++j) {
             sj[j] = __shfl_sync(0xFFFFFFFFu, my_s, half_base + j);
-            const float ru = __shfl_sync(0xFFFFFFFFu, my_ru, half_base + j);
-            const float rd = __shfl_sync(0xFFFFFFFFu, my_rd, half_base + j);
-            bad |= reciprocal_path_ok(sj[j]) ? 0u : 1u;
-            float v[8];
-            cur[j].to_float(v);
-            const uint2 codes = encode8_bracket(v, ru, rd, bad);
+            uint32_t amb4;
+            uint2 codes;
+            if constexpr (sizeof(T) == 2) {
+                const float neg_r = __shfl_sync(0xFFFFFFFFu, -my_r, half_base + j);
+                float n[8];
+                cur[j].to_neg_float(n);
+                codes = encode8_corrected(n, sj[j], neg_r);
+                amb4 = corrected_path_ok(sj[j]) ? 0u : 0xFu;
+            } else {
+                const float ru = __shfl_sync(0xFFFFFFFFu, my_r * kBracketUp, half_base + j);
+                const float rd = __shfl_sync(0xFFFFFFFFu, my_r * kBracketDown, half_base + j);
+                float v[8];
+                cur[j].to_float(v);
+                codes = encode8_bracket(v, ru, rd, amb4);
+                if (!reciprocal_path_ok(sj[j])) amb4 = 0xFu;
+            }
             const int64_t t = base + j * 16 + hw;
             if (t < total) {
                 const int64_t row = row_of(t);
                 const int64_t kb = t - row * nkb;
                 __stcs(reinterpret_cast<uint2*>(q + row * ldq + kb * 128 + hl * 8), codes);
                 if (hl == j) sa[row * sa_sm + kb * sa_skb] = sj[j];
+                amb |= amb4 << (4 * j);
             }
         }
-        if (bad != 0) {    // rare: recompute this thread's tiles with IEEE division
+        while (amb != 0) {
+            const int idx = __ffs(amb) - 1;
+            amb &= amb - 1;
+            const int j = idx >> 2;
+            float x0, x1, s = sj[0];
+            select_pair<kActTilesPerLane>(cur, idx, x0, x1);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int64_t t = base + j * 16 + hw;
-                if (t < total) {
-                    float v[8];
-                    cur[j].to_float(v);
-                    const int64_t row = row_of(t);
-                    __stcs(reinterpret_cast<uint2*>(q + row * ldq + (t - row * nkb) * 128 + hl * 8),
-                           encode8_exact(v, sj[j]));
-                }
-            }
+            for (int jj = 1; jj < kActTilesPerLane; ++jj)
+                if (j == jj) s = sj[jj];
+            const int64_t t = base + j * 16 + hw;
+            const int64_t row = row_of(t);
+            const int64_t kb = t - row * nkb;
+            *reinterpret_cast<uint16_t*>(q + row * ldq + kb * 128 + hl * 8 + 2 * (idx & 3)) =
+                static_cast<uint16_t>(encode2_exact(x0, x1, s));
         }
     }
 }

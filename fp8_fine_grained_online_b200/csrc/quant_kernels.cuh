@@ -40,6 +40,15 @@ struct Raw8<uint16_t> {  // bf16 bit patterns
             v[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
         }
     }
+    // The 8 elements negated (one IMAD / LOP3 each, like to_float).
+    __device__ __forceinline__ void to_neg_float(float (&v)[8]) const {
+        const uint32_t u[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[2 * i] = __uint_as_float((u[i] << 16) ^ 0x80000000u);
+            v[2 * i + 1] = __uint_as_float((u[i] & 0xFFFF0000u) ^ 0x80000000u);
+        }
+    }
     // max |x| of the 8 elements (exact; NaN elements are skipped), on packed
     // bf16 pairs: clear the sign bits, then lane-wise maxima.
     __device__ __forceinline__ float abs_max() const {
@@ -78,11 +87,12 @@ __device__ __forceinline__ float scale_from_amax(float amax) {
 //   |u| >= |x/s| (1 + 2^-20 - 3.1 * 2^-24) > |x/s| (1 + 2^-24) >= |RN32(x/s)|,
 //   |d| <= |x/s| (1 - 2^-20 + 3.1 * 2^-24) < |x/s| (1 - 2^-24) <= |RN32(x/s)|,
 // all with the sign of x.  E is monotone, hence when E(u) == E(d) that
-// common code is E(RN32(x/s)).  Otherwise (x/s within ~2^-20 of an E4M3
-// rounding midpoint, a fraction ~2e-5 of inputs) the codes are recomputed
-// with IEEE division.  encode8_bracket is branch free (so that the
-// multiply / convert chains of many elements interleave) and reports
-// disagreements in `bad`; callers then recompute with encode8_exact.
+// common code is E(RN32(x/s)).  Otherwise x/s lies within ~2^-20 of an
+// E4M3 rounding midpoint (~2e-5 of random fp32 inputs, but ~0.5% of bf16
+// ones, many exactly on a midpoint) and the code is recomputed with IEEE
+// division.  encode8_bracket is branch free (so that the multiply / convert
+// chains of many elements interleave) and reports disagreeing pairs; the
+// callers resolve only those pairs, one per iteration, with encode2_exact.
 // The bounds need s and 1/s to be normal fp32 numbers: tiles whose scale is
 // outside [2^-125, 2^125] use IEEE division throughout.  A quotient so small
 // that u or d is subnormal encodes to +-0 at both ends, as RN32(x/s) does;
@@ -107,18 +117,23 @@ __device__ __forceinline__ void fmul2(float& d0, float& d1, float a0, float a1, 
         : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-// Bracket-path codes of 8 values, branch free; `bad` collects the bits
-// where the two bracket ends disagree (non-zero: recompute exactly).
+// Bracket-path codes of 8 values, branch free.  Bit k of the returned
+// `amb` is set when the bracket ends disagree for elements 2k or 2k+1 (the
+// quotient lies within ~2^-20 of an E4M3 rounding midpoint).  For bf16 data
+// that is not rare: a quotient of two 8-bit mantissas times 448 lands
+// exactly on a midpoint for ~0.5% of elements, so ambiguous pairs are
+// resolved one by one (encode2_exact) rather than by recomputing tiles.
 __device__ __forceinline__ uint2 encode8_bracket(const float (&v)[8], float ru, float rd,
-                                                 uint32_t& bad) {
+                                                 uint32_t& amb) {
     uint32_t hi[4];
+    amb = 0;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         float u0, u1, d0, d1;
         fmul2(u0, u1, v[2 * k], v[2 * k + 1], ru, ru);
         fmul2(d0, d1, v[2 * k], v[2 * k + 1], rd, rd);
         hi[k] = cvt_e4m3x2(u0, u1);
-        bad |= hi[k] ^ cvt_e4m3x2(d0, d1);
+        amb |= (hi[k] != cvt_e4m3x2(d0, d1) ? 1u : 0u) << k;
     }
     uint2 out;
     out.x = hi[0] | (hi[1] << 16);
@@ -126,15 +141,95 @@ __device__ __forceinline__ uint2 encode8_bracket(const float (&v)[8], float ru, 
     return out;
 }
 
-// Codes of 8 values through IEEE fp32 division (the definition).
-__device__ __forceinline__ uint2 encode8_exact(const float (&v)[8], float s) {
-    float d[8];
+// ---------------------------------------------------------------------------
+// bf16 inputs: a corrected quotient.  With r = RN32(1 / s) and n = -x:
+//   q0 = RN32(n (-r)) = RN32(x r),
+//   t  = RN32(q0 s + n) = RN32(q0 s - x)   (FMA; exact),
+//   q1 = RN32(t (-r) + q0)                 (FMA),
+// and the code is E(q1).  For every bf16 x with |x| <= amax and every bf16
+// amax whose scale s = RN32(amax / 448) lies in [2^-100, 2^125], E(q1) equals
+// E(RN32(x / s)), signs and signed zeros included: checked exhaustively over
+// all such pairs (about 1e9), which is a complete proof for bf16 data
+// because a tile's elements are bf16 values no larger than its amax.  (q1
+// itself is not always the correctly rounded quotient, but where it
+// differs the two lie on the same side of every E4M3 rounding boundary.)
+// Working on n = -x keeps x = -0 at -0 through both FMAs (q0 - t r with
+// q0 = -0 and t = +0 is -0), and costs nothing: the bf16 -> fp32 unpack of
+// -x is as cheap as that of x.  Three packed operations and one convert per
+// pair, branch free.  fp32 inputs, which the exhaustive check does not
+// cover, take the bracket path below.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ bool corrected_path_ok(float s) {
+    return s >= 0x1p-100f && s <= 0x1p125f;
+}
+
+// n: the 8 inputs negated; neg_r = -RN32(1 / s).
+__device__ __forceinline__ uint2 encode8_corrected(const float (&n)[8], float s, float neg_r) {
+    uint32_t c[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) d[i] = __fdiv_rn(v[i], s);
+    for (int k = 0; k < 4; ++k) {
+        float q0, q1;
+        fmul2(q0, q1, n[2 * k], n[2 * k + 1], neg_r, neg_r);
+        float t0 = n[2 * k], t1 = n[2 * k + 1];
+        ffma2_scalar(t0, t1, s, q0, q1);          // q0 s - x, exact
+        ffma2_scalar(q0, q1, neg_r, t0, t1);      // q0 - t r
+        c[k] = cvt_e4m3x2(q0, q1);
+    }
     uint2 out;
-    out.x = cvt_e4m3x2(d[0], d[1]) | (cvt_e4m3x2(d[2], d[3]) << 16);
-    out.y = cvt_e4m3x2(d[4], d[5]) | (cvt_e4m3x2(d[6], d[7]) << 16);
+    out.x = c[0] | (c[1] << 16);
+    out.y = c[2] | (c[3] << 16);
     return out;
+}
+
+// Codes of 2 values through IEEE fp32 division (the definition); the
+// first value in the low byte.
+__device__ __forceinline__ uint32_t encode2_exact(float x0, float x1, float s) {
+    return cvt_e4m3x2(__fdiv_rn(x0, s), __fdiv_rn(x1, s));
+}
+
+// Pair `idx` = 4 j + k (elements 2k, 2k+1 of raw[j]) as fp32, selected
+// without indexing registers dynamically.
+template <int kJ>
+__device__ __forceinline__ void select_pair(const Raw8<uint16_t> (&raw)[kJ], int idx, float& x0,
+                                            float& x1) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int j = 0; j < kJ; ++j) {
+        const uint32_t u[4] = {raw[j].a.x, raw[j].a.y, raw[j].a.z, raw[j].a.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (idx == 4 * j + k) w = u[k];
+    }
+    x0 = __uint_as_float(w << 16);
+    x1 = __uint_as_float(w & 0xFFFF0000u);
+}
+
+template <int kJ>
+__device__ __forceinline__ void select_pair(const Raw8<float> (&raw)[kJ], int idx, float& x0,
+                                            float& x1) {
+    x0 = 0.0f;
+    x1 = 0.0f;
+#pragma unroll
+    for (int j = 0; j < kJ; ++j) {
+        const float u[8] = {raw[j].a.x, raw[j].a.y, raw[j].a.z, raw[j].a.w,
+                            raw[j].b.x, raw[j].b.y, raw[j].b.z, raw[j].b.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (idx == 4 * j + k) {
+                x0 = u[2 * k];
+                x1 = u[2 * k + 1];
+            }
+    }
+}
+
+// Replace the 16-bit code pair k (bytes 2k, 2k+1) of an 8-code group.
+__device__ __forceinline__ void patch_pair(uint2& codes, int k, uint32_t c16) {
+    const uint32_t sh = (k & 1) * 16;
+    const uint32_t keep = ~(0xFFFFu << sh);
+    if (k < 2)
+        codes.x = (codes.x & keep) | (c16 << sh);
+    else
+        codes.y = (codes.y & keep) | (c16 << sh);
 }
 
 // floor(n / d) for 0 <= n < 2^31 and a fixed d >= 1, by multiplication:

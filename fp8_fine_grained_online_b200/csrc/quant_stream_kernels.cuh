@@ -1,22 +1,21 @@
-// quant_stream_kernels.cuh -- online fine-grained E4M3 quantization streamed
+// quant_stream_kernels.cuh -- online 128x128 weight quantization streamed
 // through shared memory by TMA.
 //
-// Activations: every 1x128 tile of x [M, K] gets scale = amax / 448;
-// weights: every 128x128 block of w [K, N] gets scale = amax / 448
-// (codingmall.com "Kan du förklara rollen för FP8 precision i
-// träningsprocessen för DeepSeek-V3", "Finkornig kvantisering",
+// Every 128x128 block of w [K, N] gets scale = amax / 448 and codes
+// E4M3_RNE_satfinite(w / scale), bit-exact to IEEE fp32 division (see
+// encode8_bracket) (codingmall.com "Kan du förklara rollen för FP8 precision
+// i träningsprocessen för DeepSeek-V3", "Finkornig kvantisering",
 // "Online-kvantisering"; holysheep.ai "FP8 混精度训练 DeepSeek 671B" (zh),
-// 2.2).  Codes are E4M3_RNE_satfinite(x / scale), bit-exact to IEEE fp32
-// division (see encode_pair).
+// 2.2).  Output [K, N] as given, or transposed to [N, K] (K contiguous, the
+// GEMM's B operand layout).
 //
-// Both are HBM-bound.  One persistent CTA per SM with two groups of 8
-// warps.  Group g takes the CTA's boxes g, g+2, ... of 128x128 input
-// elements; each group owns two shared-memory slots (one for fp32 input)
-// that its first thread fills by TMA.  For every box the group copies its
-// slot to registers, meets at a group barrier, and the slot is refilled with
-// the group's box two ahead while the group computes the scales, encodes and
-// writes codes and scales; so HBM reads overlap the arithmetic of both
-// groups.
+// HBM-bound.  One persistent CTA per SM with two groups of 8 warps.  Group
+// g takes the CTA's boxes g, g+2, ... of 128x128 input elements; each group
+// owns two shared-memory slots (one for fp32 input) that its first thread
+// fills by TMA.  A block is read from shared memory twice (amax pass, then
+// encode pass); the slot is refilled with the group's box two ahead as soon
+// as the group has taken its second half into registers, so HBM reads
+// overlap the arithmetic of both groups.
 //
 // Consumer thread (kq = t / 16, c = t % 16) of its group holds rows
 // {4kq .. 4kq+3, 64+4kq .. 64+4kq+3} of the box, columns [8c, 8c+8).
@@ -31,7 +30,7 @@
 
 namespace fp8fg {
 
-enum QuantMode { kQuantAct = 0, kQuantWeight = 1, kQuantWeightT = 2 };
+enum QuantMode { kQuantWeight = 1, kQuantWeightT = 2 };
 
 constexpr int kQsGroups = 2;                 // consumer groups of 8 warps
 constexpr int kQsThreads = kQsGroups * 256;
@@ -120,40 +119,6 @@ __device__ __forceinline__ void transpose4x4_bytes(uint32_t r0, uint32_t r1, uin
     w[3] = __byte_perm(t1, t3, 0x7632);
 }
 
-// Per-row amax of 8 rows held by a half-warp (16 lanes x 8 elements per
-// row): every lane gets all eight row maxima.
-template <typename T>
-__device__ __forceinline__ void row_amax8(const Raw8<T> (&raw)[8], float (&amax)[8]);
-
-// bf16: a row maximum is an exact bf16 value, so two rows travel in one
-// register and are reduced with packed bf16 maxima.
-template <>
-__device__ __forceinline__ void row_amax8<uint16_t>(const Raw8<uint16_t> (&raw)[8],
-                                                    float (&amax)[8]) {
-#pragma unroll
-    for (int j = 0; j < 8; j += 2) {
-        const uint32_t a0 = __float_as_uint(raw[j].abs_max()) >> 16;        // bf16 bits
-        const uint32_t a1 = __float_as_uint(raw[j + 1].abs_max()) & 0xFFFF0000u;
-        uint32_t m = a0 | a1;
-#pragma unroll
-        for (int off = 8; off > 0; off >>= 1)
-            m = bf16x2_max(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
-        amax[j] = __uint_as_float(m << 16);
-        amax[j + 1] = __uint_as_float(m & 0xFFFF0000u);
-    }
-}
-
-template <>
-__device__ __forceinline__ void row_amax8<float>(const Raw8<float> (&raw)[8], float (&amax)[8]) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        float a = raw[j].abs_max();
-#pragma unroll
-        for (int off = 8; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
-        amax[j] = a;
-    }
-}
-
 template <typename T, int kMode>
 __global__ void __launch_bounds__(kQsThreads, 1)
     quant_stream_kernel(const __grid_constant__ CUtensorMap tm_in, const QsParams p) {
@@ -224,142 +189,105 @@ __global__ void __launch_bounds__(kQsThreads, 1)
         const int64_t br = box / p.nbc;
         const int64_t bc = box - br * p.nbc;
 
-        if (kMode == kQuantAct) {
-            // One 1x128 tile per row: the 16 lanes of a half-warp share a row.
-            // Lane c computes the scale of row slot (c & 7) once; the half-
-            // warp shares the eight scales by shuffle.
-            const int half_base = lane & 16;
-            Raw8<T> raw[8];
+        // One scale for the whole 128x128 box: an amax pass over the box
+        // in shared memory, a block reduction, then an encode pass.
+        float a = 0.0f;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) load_raw_smem<T>(row_ptr(j), c, raw[j]);
-            if (!release_stage()) break;
-            float amax[8];
-            row_amax8<T>(raw, amax);
-            float my_amax = amax[0];
+        for (int j = 0; j < 8; ++j) {
+            Raw8<T> r;
+            load_raw_smem<T>(row_ptr(j), c, r);
+            a = fmaxf(a, r.abs_max());
+        }
 #pragma unroll
-            for (int j = 1; j < 8; ++j)
-                if ((c & 7) == j) my_amax = amax[j];
-            const float my_s = scale_from_amax(my_amax);
-            const float my_r = __frcp_rn(my_s);
-            const float my_ru = my_r * kBracketUp;
-            const float my_rd = my_r * kBracketDown;
-            // Codes are stored row by row; in the rare case of a bracket
-            // disagreement (or a scale off the reciprocal path) the thread
-            // recomputes its rows with IEEE division and overwrites them.
-            float sj[8];
-            uint32_t bad = 0;
-            uint8_t* qrow0 = p.q + (br * 128) * p.ldq + bc * 128 + c * 8;
+        for (int off = 16; off > 0; off >>= 1)
+            a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+        const int par = static_cast<int>((i / kQsGroups) & 1);
+        if (lane == 0) tail->red[g][par][wg] = a;
+        if (!group_sync(&tail->gbar[g], gbar_uses, lane, abort_flag)) break;
+        a = tail->red[g][par][0];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                sj[j] = __shfl_sync(0xFFFFFFFFu, my_s, half_base + j);
-                const float ru = __shfl_sync(0xFFFFFFFFu, my_ru, half_base + j);
-                const float rd = __shfl_sync(0xFFFFFFFFu, my_rd, half_base + j);
-                bad |= reciprocal_path_ok(sj[j]) ? 0u : 1u;
-                float v[8];
-                raw[j].to_float(v);
-                const uint2 codes = encode8_bracket(v, ru, rd, bad);
-                const int r = row_in_box(j);
-                if (br * 128 + r < p.rows) {
-                    __stcs(reinterpret_cast<uint2*>(qrow0 + r * p.ldq), codes);
-                    if (c == j) p.s[(br * 128 + r) * p.s_stride_r + bc * p.s_stride_c] = sj[j];
-                }
-            }
-            if (bad != 0) {
+        for (int w = 1; w < 8; ++w) a = fmaxf(a, tail->red[g][par][w]);
+        const float s = scale_from_amax(a);
+        const float rcp = __frcp_rn(s);
+        const float ru = rcp * kBracketUp;
+        const float rd = rcp * kBracketDown;
+        const bool off_path = sizeof(T) == 2 ? !corrected_path_ok(s) : !reciprocal_path_ok(s);
+        if (t == 0) p.s[br * p.s_stride_r + bc * p.s_stride_c] = s;
+        uint32_t(*tb)[33] = tail->tbuf[g];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    float v[8];
-                    raw[j].to_float(v);
-                    const int r = row_in_box(j);
-                    if (br * 128 + r < p.rows)
-                        __stcs(reinterpret_cast<uint2*>(qrow0 + r * p.ldq), encode8_exact(v, sj[j]));
-                }
-            }
-        } else {
-            // One scale for the whole 128x128 box: an amax pass over the box
-            // in shared memory, a block reduction, then an encode pass.
-            float a = 0.0f;
+        for (int h4 = 0; h4 < 2; ++h4) {
+            Raw8<T> raw[4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                Raw8<T> r;
-                load_raw_smem<T>(row_ptr(j), c, r);
-                a = fmaxf(a, r.abs_max());
-            }
+            for (int jj = 0; jj < 4; ++jj) load_raw_smem<T>(row_ptr(h4 * 4 + jj), c, raw[jj]);
+            if (h4 == 1 && !release_stage()) break;
+            // bf16: corrected quotient.  fp32: bracket; pairs whose ends
+            // disagree (bit 4 jj + k) are recomputed with IEEE division, one
+            // per iteration, as are all pairs of a block whose scale is off
+            // the fast path.
+            uint2 codes[4];
+            uint32_t amb = 0;
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1)
-                a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
-            const int par = static_cast<int>((i / kQsGroups) & 1);
-            if (lane == 0) tail->red[g][par][wg] = a;
-            if (!group_sync(&tail->gbar[g], gbar_uses, lane, abort_flag)) break;
-            a = tail->red[g][par][0];
-#pragma unroll
-            for (int w = 1; w < 8; ++w) a = fmaxf(a, tail->red[g][par][w]);
-            const float s = scale_from_amax(a);
-            const float rcp = __frcp_rn(s);
-            const float ru = rcp * kBracketUp;
-            const float rd = rcp * kBracketDown;
-            const uint32_t off_path = reciprocal_path_ok(s) ? 0u : 1u;
-            if (t == 0) p.s[br * p.s_stride_r + bc * p.s_stride_c] = s;
-            uint32_t(*tb)[33] = tail->tbuf[g];
-#pragma unroll
-            for (int h4 = 0; h4 < 2; ++h4) {
-                Raw8<T> raw[4];
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) load_raw_smem<T>(row_ptr(h4 * 4 + jj), c, raw[jj]);
-                if (h4 == 1 && !release_stage()) break;
-                uint2 codes[4];
-                uint32_t bad = off_path;
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
+            for (int jj = 0; jj < 4; ++jj) {
+                if constexpr (sizeof(T) == 2) {
+                    float n[8];
+                    raw[jj].to_neg_float(n);
+                    codes[jj] = encode8_corrected(n, s, -rcp);
+                } else {
                     float v[8];
                     raw[jj].to_float(v);
-                    codes[jj] = encode8_bracket(v, ru, rd, bad);
-                }
-                if (bad != 0) {    // rare: recompute these rows exactly
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        float v[8];
-                        raw[jj].to_float(v);
-                        codes[jj] = encode8_exact(v, s);
-                    }
-                }
-                if (kMode == kQuantWeight) {
-                    uint8_t* dst = p.q + (br * 128) * p.ldq + bc * 128 + c * 8;
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj)
-                        __stcs(reinterpret_cast<uint2*>(dst + row_in_box(h4 * 4 + jj) * p.ldq),
-                               codes[jj]);
-                } else {
-                    // Transposed output [N, K]: per column n, the codes of rows
-                    // 4kq..4kq+3 (+64 h4) form one word of tbuf[n][k/4]; a 4x4
-                    // byte transpose of each half of the four rows' codes.
-                    uint32_t wx[4], wy[4];
-                    transpose4x4_bytes(codes[0].x, codes[1].x, codes[2].x, codes[3].x, wx);
-                    transpose4x4_bytes(codes[0].y, codes[1].y, codes[2].y, codes[3].y, wy);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        tb[c * 8 + e][h4 * 16 + kq] = wx[e];
-                        tb[c * 8 + 4 + e][h4 * 16 + kq] = wy[e];
-                    }
+                    uint32_t amb4;
+                    codes[jj] = encode8_bracket(v, ru, rd, amb4);
+                    amb |= amb4 << (4 * jj);
                 }
             }
-            if (*abort_flag) break;
-            if (kMode == kQuantWeightT) {
-                if (!group_sync(&tail->gbar[g], gbar_uses, lane, abort_flag)) break;
-                const int n = t >> 1;
-                const int part = t & 1;
-                uint8_t* dst = p.q + (bc * 128 + n) * p.ldq + br * 128 + part * 64;
+            if (off_path) amb = 0xFFFFu;
+            while (amb != 0) {
+                const int idx = __ffs(amb) - 1;
+                amb &= amb - 1;
+                float x0, x1;
+                select_pair<4>(raw, idx, x0, x1);
+                const uint32_t c16 = encode2_exact(x0, x1, s);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint4 o;
-                    o.x = tb[n][part * 16 + j * 4 + 0];
-                    o.y = tb[n][part * 16 + j * 4 + 1];
-                    o.z = tb[n][part * 16 + j * 4 + 2];
-                    o.w = tb[n][part * 16 + j * 4 + 3];
-                    __stcs(reinterpret_cast<uint4*>(dst) + j, o);
-                }
-                // tbuf is rewritten for the next box
-                if (!group_sync(&tail->gbar[g], gbar_uses, lane, abort_flag)) break;
+                for (int jj = 0; jj < 4; ++jj)
+                    if ((idx >> 2) == jj) patch_pair(codes[jj], idx & 3, c16);
             }
+            if (kMode == kQuantWeight) {
+                uint8_t* dst = p.q + (br * 128) * p.ldq + bc * 128 + c * 8;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj)
+                    __stcs(reinterpret_cast<uint2*>(dst + row_in_box(h4 * 4 + jj) * p.ldq),
+                           codes[jj]);
+            } else {
+                // Transposed output [N, K]: per column n, the codes of rows
+                // 4kq..4kq+3 (+64 h4) form one word of tbuf[n][k/4]; a 4x4
+                // byte transpose of each half of the four rows' codes.
+                uint32_t wx[4], wy[4];
+                transpose4x4_bytes(codes[0].x, codes[1].x, codes[2].x, codes[3].x, wx);
+                transpose4x4_bytes(codes[0].y, codes[1].y, codes[2].y, codes[3].y, wy);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    tb[c * 8 + e][h4 * 16 + kq] = wx[e];
+                    tb[c * 8 + 4 + e][h4 * 16 + kq] = wy[e];
+                }
+            }
+        }
+        if (*abort_flag) break;
+        if (kMode == kQuantWeightT) {
+            if (!group_sync(&tail->gbar[g], gbar_uses, lane, abort_flag)) break;
+            const int n = t >> 1;
+            const int part = t & 1;
+            uint8_t* dst = p.q + (bc * 128 + n) * p.ldq + br * 128 + part * 64;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint4 o;
+                o.x = tb[n][part * 16 + j * 4 + 0];
+                o.y = tb[n][part * 16 + j * 4 + 1];
+                o.z = tb[n][part * 16 + j * 4 + 2];
+                o.w = tb[n][part * 16 + j * 4 + 3];
+                __stcs(reinterpret_cast<uint4*>(dst) + j, o);
+            }
+            // tbuf is rewritten for the next box
+            if (!group_sync(&tail->gbar[g], gbar_uses, lane, abort_flag)) break;
         }
     }
     // After an abandoned wait a refill may still be in flight: let it land

@@ -63,3 +63,26 @@ def assert_gemm_within_bound(c_gpu, c_ref, T, out_dtype):
                              "T %r (err/bound %.3g)" % (bad.sum(), bad.size, i, c[i], c_ref[i],
                                                         T[i], (err / bound)[i]))
     return float(np.max(err / bound))
+
+
+def bf16_quotient_sweep(amax_exps=(35, 36, 37, 100, 127, 160, 254), depth=20):
+    """Structured bf16 inputs covering every (amax, x) mantissa pair.
+
+    For each amax = 2^(e-127) (1 + m/128) (m = 0..127, e in amax_exps) the
+    list holds amax first, then every bf16 x of either sign with exponent
+    field in [e - depth, e] and |x| <= amax.  Quotients x / s reach down to
+    amax 2^-(depth+1) / s, below the smallest E4M3 midpoint (2^-10).
+    Returns a list of uint16 arrays (bf16 bit patterns), one per amax."""
+    out = []
+    mant = np.arange(128, dtype=np.uint16)
+    for e in amax_exps:
+        lo = max(1, e - depth)
+        for m in range(128):
+            amax = np.uint16((e << 7) | m)
+            xs = []
+            for ex in range(lo, e + 1):
+                mm = mant if ex < e else mant[:m + 1]
+                xs.append((np.uint16(ex) << 7) | mm)
+            mag = np.concatenate(xs).astype(np.uint16)
+            out.append(np.concatenate([[amax], mag, mag | np.uint16(0x8000)]).astype(np.uint16))
+    return out

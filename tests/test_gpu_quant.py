@@ -180,3 +180,52 @@ def test_quant_bandwidth_workload_sampled(cuda_lib, orc):
         qo, sbo = orc.quantize_weight_128x128(to_oracle(blk), transpose_out=True)
         assert_codes_equal(np_u8(qw[nb * 128:(nb + 1) * 128, kb * 128:(kb + 1) * 128]), qo)
         assert_scales_equal(sb[kb:kb + 1, nb:nb + 1].cpu().numpy(), sbo)
+
+
+def _bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits, dtype=np.uint16).view(np.int16)) \
+        .view(torch.bfloat16)
+
+
+def test_act_bf16_quotient_sweep(cuda_lib, orc):
+    """Every bf16 (amax, x) mantissa pair over 21 exponent steps, at amax
+    exponents that put the scale near the bottom of the fast path, just
+    below it, and across the range: codes of the fast quotient equal those
+    of IEEE division."""
+    from _util import bf16_quotient_sweep
+    rows = []
+    for lst in bf16_quotient_sweep():
+        amax, xs = lst[0], lst[1:]
+        for i in range(0, len(xs), 127):
+            row = np.zeros(128, dtype=np.uint16)
+            row[0] = amax
+            chunk = xs[i:i + 127]
+            row[1:1 + len(chunk)] = chunk
+            rows.append(row)
+    bits = np.stack(rows)
+    x = _bf16(bits)
+    q, sa = cuda_lib.fp8_quantize_act_1x128(x.cuda())
+    qo, sao = orc.quantize_act_1x128(bits)
+    assert_scales_equal(sa.cpu().numpy(), sao)
+    assert_codes_equal(np_u8(q), qo)
+
+
+@pytest.mark.parametrize("transpose_out", [False, True])
+def test_weight_bf16_quotient_sweep(cuda_lib, orc, transpose_out):
+    """The same sweep through the 128x128 weight quantizer: one amax (and
+    all its x) per block."""
+    from _util import bf16_quotient_sweep
+    lists = bf16_quotient_sweep()
+    nb = len(lists)                       # 896 blocks: 28 x 32
+    kb_n, nb_n = 28, 32
+    assert nb == kb_n * nb_n
+    w = np.zeros((kb_n * 128, nb_n * 128), dtype=np.uint16)
+    for i, lst in enumerate(lists):
+        blk = np.zeros(128 * 128, dtype=np.uint16)
+        blk[:len(lst)] = lst
+        r, c = divmod(i, nb_n)
+        w[r * 128:(r + 1) * 128, c * 128:(c + 1) * 128] = blk.reshape(128, 128)
+    q, sb = cuda_lib.fp8_quantize_weight_128x128(_bf16(w).cuda(), transpose_out=transpose_out)
+    qo, sbo = orc.quantize_weight_128x128(w, transpose_out=transpose_out)
+    assert_scales_equal(sb.cpu().numpy(), sbo)
+    assert_codes_equal(np_u8(q), qo)
