@@ -488,6 +488,23 @@ CPU_BASELINE_SAMPLE = {"ffn": (128, 12), "quant": (64, 24), "moe": (128, 6), "dg
 
 # ----------------------------------------------------------------------------- timing
 
+def max_over_ranks(ms, world, device):
+    """The slowest rank's time: every rank contributes its own device-timed
+    milliseconds and all of them get the maximum (one collective, taken in
+    the same order on every rank)."""
+    if world <= 1:
+        return float(ms)
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_rate(world, work_per_step, steps, max_ms):
+    """Whole-job throughput of `world` replicas that each did `steps` steps
+    of `work_per_step` units, timed as the slowest rank (weak scaling)."""
+    return world * work_per_step * steps / (max_ms / 1e3)
+
+
 def run_ours(args, rank, world, local_rank):
     import fp8_fine_grained_online_b200 as fp8
     device = "cuda:%d" % local_rank
@@ -521,11 +538,7 @@ def run_ours(args, rank, world, local_rank):
     wall = time.perf_counter() - wall0
     barrier()
     clk = clocks.stop()
-    elapsed_ms = start.elapsed_time(stop)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(start.elapsed_time(stop), world, device)
     dev_err = fp8.fp8_get_device_error()
 
     per_kernel = {}
@@ -548,12 +561,8 @@ def run_ours(args, rank, world, local_rank):
             wl.e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=device)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": round(world * wl.work_per_step() * n_e2e / (e_ms / 1e3) / scale(wl), 3),
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+        e2e = {"value": round(aggregate_rate(world, wl.work_per_step(), n_e2e, e_ms) / scale(wl), 3),
                "unit": wl.unit, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": n_e2e}
     return wl, elapsed_ms, per_kernel, clk, e2e, wall, dev_err
@@ -658,7 +667,7 @@ def main():
         if rank != 0:
             return
         peaks, peak_src = load_peaks()
-        value = world * wl.work_per_step() * args.steps / (elapsed_ms / 1e3) / scale(wl)
+        value = aggregate_rate(world, wl.work_per_step(), args.steps, elapsed_ms) / scale(wl)
         kernels = {}
         for k, ms in per_kernel.items():
             r = roofline_entry(wl, k, ms, peaks, peak_src)
