@@ -505,11 +505,20 @@ def aggregate_rate(world, work_per_step, steps, max_ms):
     return world * work_per_step * steps / (max_ms / 1e3)
 
 
+def make_workload(args, fp8, device):
+    """The workload object; --moe-experts E shrinks the MoE workload to E
+    experts and 32 E tokens (same rows per expert), for profiler captures
+    that must stay small."""
+    if args.workload == "moe" and args.moe_experts != 256:
+        return MoE(fp8, device, tokens=32 * args.moe_experts, experts=args.moe_experts)
+    return WORKLOADS[args.workload](fp8, device)
+
+
 def run_ours(args, rank, world, local_rank):
     import fp8_fine_grained_online_b200 as fp8
     device = "cuda:%d" % local_rank
     torch.cuda.set_device(local_rank)
-    wl = WORKLOADS[args.workload](fp8, device)
+    wl = make_workload(args, fp8, device)
     stream = torch.cuda.current_stream()
     nk = len(wl.kernels)
 
@@ -619,6 +628,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="ffn")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--moe-experts", type=int, default=256,
+                    help="MoE workload only: number of experts (tokens = 32 x experts)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

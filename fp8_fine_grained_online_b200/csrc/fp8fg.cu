@@ -77,12 +77,14 @@ fp8_status_t current_device(int* dev_out, int* sms_out) {
                     }
                 }
                 const void* qs_bf16[] = {
+                    reinterpret_cast<const void*>(&quant_stream_kernel<uint16_t, kQuantAct>),
                     reinterpret_cast<const void*>(&quant_stream_kernel<uint16_t, kQuantWeight>),
                     reinterpret_cast<const void*>(&quant_stream_kernel<uint16_t, kQuantWeightT>)};
                 const void* qs_f32[] = {
+                    reinterpret_cast<const void*>(&quant_stream_kernel<float, kQuantAct>),
                     reinterpret_cast<const void*>(&quant_stream_kernel<float, kQuantWeight>),
                     reinterpret_cast<const void*>(&quant_stream_kernel<float, kQuantWeightT>)};
-                for (int i = 0; i < 2; ++i) {
+                for (int i = 0; i < 3; ++i) {
                     if (cudaFuncSetAttribute(qs_bf16[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(quant_stream_smem_bytes<uint16_t>())) !=
                             cudaSuccess ||
@@ -167,6 +169,9 @@ inline fp8_status_t launch_status() {
     return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
+// Activation quantization: TMA-streamed boxes (true) or register tiles (false).
+constexpr bool kActUseStream = true;
+
 int elem_size_in(fp8_in_t t) { return t == FP8_IN_BF16 ? 2 : (t == FP8_IN_FP32 ? 4 : 0); }
 int elem_size_out(fp8_out_t t) { return t == FP8_OUT_BF16 ? 2 : (t == FP8_OUT_FP32 ? 4 : 0); }
 
@@ -234,10 +239,12 @@ fp8_status_t launch_quant_stream(const void* in, fp8_in_t t, int64_t ld, const Q
                         static_cast<uint64_t>(ld)))
         return FP8_ERR_CUDA;
     if (t == FP8_IN_BF16) {
+        if (mode == kQuantAct) return launch_quant_stream_t<uint16_t, kQuantAct>(map, p, sms, stream);
         if (mode == kQuantWeight)
             return launch_quant_stream_t<uint16_t, kQuantWeight>(map, p, sms, stream);
         return launch_quant_stream_t<uint16_t, kQuantWeightT>(map, p, sms, stream);
     }
+    if (mode == kQuantAct) return launch_quant_stream_t<float, kQuantAct>(map, p, sms, stream);
     if (mode == kQuantWeight) return launch_quant_stream_t<float, kQuantWeight>(map, p, sms, stream);
     return launch_quant_stream_t<float, kQuantWeightT>(map, p, sms, stream);
 }
@@ -281,6 +288,14 @@ fp8_status_t fp8_quantize_act_1x128(const void* x, fp8_in_t x_type, int64_t M, i
     int dev, sms;
     fp8_status_t st = current_device(&dev, &sms);
     if (st != FP8_OK) return st;
+    if (kActUseStream) {
+        QsParams p{};
+        p.rows = M; p.cols = K;
+        p.nbr = (M + 127) / 128; p.nbc = K / 128;
+        p.q = q; p.ldq = ldq;
+        p.s = sa; p.s_stride_r = sa_stride_m; p.s_stride_c = sa_stride_kb;
+        return launch_quant_stream(x, x_type, ldx, p, kQuantAct, sms, stream);
+    }
     const int64_t nkb = K / 128;
     const int64_t tiles = M * nkb;
     const int64_t grid = grid_for((tiles + kActTilesPerStep - 1) / kActTilesPerStep, sms, kActMinBlocks);

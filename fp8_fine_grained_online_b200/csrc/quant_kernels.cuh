@@ -76,6 +76,49 @@ __device__ __forceinline__ float scale_from_amax(float amax) {
     return s == 0.0f ? 1.0f : s;
 }
 
+// amax[j] = max |x| over tile j of the half-warp (all 16 lanes get it).
+template <typename T, int kJ>
+__device__ __forceinline__ void half_warp_amax(const Raw8<T> (&raw)[kJ], float (&amax)[kJ]);
+
+// bf16: a tile maximum is an exact bf16 value, so two tiles travel in one
+// register and are reduced with packed bf16 maxima.
+template <int kJ>
+__device__ __forceinline__ void half_warp_amax_bf16(const Raw8<uint16_t> (&raw)[kJ],
+                                                    float (&amax)[kJ]) {
+    static_assert(kJ % 2 == 0, "tiles are reduced in pairs");
+#pragma unroll
+    for (int j = 0; j < kJ; j += 2) {
+        const uint32_t a0 = __float_as_uint(raw[j].abs_max()) >> 16;
+        const uint32_t a1 = __float_as_uint(raw[j + 1].abs_max()) & 0xFFFF0000u;
+        uint32_t m = a0 | a1;
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1)
+            m = bf16x2_max(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+        amax[j] = __uint_as_float(m << 16);
+        amax[j + 1] = __uint_as_float(m & 0xFFFF0000u);
+    }
+}
+
+template <int kJ>
+__device__ __forceinline__ void half_warp_amax_f32(const Raw8<float> (&raw)[kJ],
+                                                   float (&amax)[kJ]) {
+#pragma unroll
+    for (int j = 0; j < kJ; ++j) {
+        float a = raw[j].abs_max();
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+        amax[j] = a;
+    }
+}
+
+template <typename T, int kJ>
+__device__ __forceinline__ void half_warp_amax(const Raw8<T> (&raw)[kJ], float (&amax)[kJ]) {
+    if constexpr (sizeof(T) == 2)
+        half_warp_amax_bf16<kJ>(raw, amax);
+    else
+        half_warp_amax_f32<kJ>(raw, amax);
+}
+
 // ---------------------------------------------------------------------------
 // E4M3 code of the IEEE fp32 quotient x / s, without a division per element.
 //

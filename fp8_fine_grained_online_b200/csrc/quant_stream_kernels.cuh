@@ -30,7 +30,7 @@
 
 namespace fp8fg {
 
-enum QuantMode { kQuantWeight = 1, kQuantWeightT = 2 };
+enum QuantMode { kQuantAct = 0, kQuantWeight = 1, kQuantWeightT = 2 };
 
 constexpr int kQsGroups = 2;                 // consumer groups of 8 warps
 constexpr int kQsThreads = kQsGroups * 256;
@@ -47,7 +47,7 @@ struct QsSmemTail {
     uint64_t full[4];                  // slot filled (TMA bytes)
     uint64_t gbar[kQsGroups];          // per-group barrier (8 warp arrivals)
     float red[kQsGroups][2][8];        // [group][block parity][warp]
-    uint32_t tbuf[kQsGroups][128][33]; // [group][n][k/4], transposed codes
+    uint32_t tbuf[kQsGroups][2][128][33]; // [group][box parity][n][k/4 swizzled], transposed codes
     int abort_flag;
 };
 
@@ -189,6 +189,69 @@ __global__ void __launch_bounds__(kQsThreads, 1)
         const int64_t br = box / p.nbc;
         const int64_t bc = box - br * p.nbc;
 
+        if constexpr (kMode == kQuantAct) {
+            // One 1x128 tile per row: the 16 lanes of a half-warp share 8
+            // rows.  Lane c computes the scale of row slot (c & 7) once and
+            // the half-warp shares the eight scales by shuffle.
+            const int half_base = lane & 16;
+            Raw8<T> raw[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) load_raw_smem<T>(row_ptr(j), c, raw[j]);
+            if (!release_stage()) break;
+            float amax[8];
+            half_warp_amax<T, 8>(raw, amax);
+            float my_amax = amax[0];
+#pragma unroll
+            for (int j = 1; j < 8; ++j)
+                if ((c & 7) == j) my_amax = amax[j];
+            const float my_s = scale_from_amax(my_amax);
+            const float my_r = __frcp_rn(my_s);
+            // bf16: corrected quotient; fp32: bracket, with its ambiguous
+            // pairs (bit 4j + k) recomputed by IEEE division afterwards, as
+            // are all pairs of a row whose scale is off the fast path.
+            float sj[8];
+            uint32_t amb = 0;
+            uint8_t* qrow0 = p.q + (br * 128) * p.ldq + bc * 128 + c * 8;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                sj[j] = __shfl_sync(0xFFFFFFFFu, my_s, half_base + j);
+                uint32_t amb4;
+                uint2 codes;
+                if constexpr (sizeof(T) == 2) {
+                    const float neg_r = __shfl_sync(0xFFFFFFFFu, -my_r, half_base + j);
+                    float n[8];
+                    raw[j].to_neg_float(n);
+                    codes = encode8_corrected(n, sj[j], neg_r);
+                    amb4 = corrected_path_ok(sj[j]) ? 0u : 0xFu;
+                } else {
+                    const float ru = __shfl_sync(0xFFFFFFFFu, my_r * kBracketUp, half_base + j);
+                    const float rd = __shfl_sync(0xFFFFFFFFu, my_r * kBracketDown, half_base + j);
+                    float v[8];
+                    raw[j].to_float(v);
+                    codes = encode8_bracket(v, ru, rd, amb4);
+                    if (!reciprocal_path_ok(sj[j])) amb4 = 0xFu;
+                }
+                const int r = row_in_box(j);
+                if (br * 128 + r < p.rows) {
+                    __stcs(reinterpret_cast<uint2*>(qrow0 + r * p.ldq), codes);
+                    if (c == j) p.s[(br * 128 + r) * p.s_stride_r + bc * p.s_stride_c] = sj[j];
+                    amb |= amb4 << (4 * j);
+                }
+            }
+            while (amb != 0) {
+                const int idx = __ffs(amb) - 1;
+                amb &= amb - 1;
+                const int j = idx >> 2;
+                float x0, x1, sv = sj[0];
+                select_pair<8>(raw, idx, x0, x1);
+#pragma unroll
+                for (int jj = 1; jj < 8; ++jj)
+                    if (j == jj) sv = sj[jj];
+                *reinterpret_cast<uint16_t*>(qrow0 + row_in_box(j) * p.ldq + 2 * (idx & 3)) =
+                    static_cast<uint16_t>(encode2_exact(x0, x1, sv));
+            }
+            continue;
+        } else {
         // One scale for the whole 128x128 box: an amax pass over the box
         // in shared memory, a block reduction, then an encode pass.
         float a = 0.0f;
@@ -213,7 +276,12 @@ __global__ void __launch_bounds__(kQsThreads, 1)
         const float rd = rcp * kBracketDown;
         const bool off_path = sizeof(T) == 2 ? !corrected_path_ok(s) : !reciprocal_path_ok(s);
         if (t == 0) p.s[br * p.s_stride_r + bc * p.s_stride_c] = s;
-        uint32_t(*tb)[33] = tail->tbuf[g];
+        uint32_t(*tb)[33] = tail->tbuf[g][par];
+        // Word w of row n sits at column (w + 2 (n / 8)) mod 32 of a 33-word
+        // row: the stores below (n = 8c + e, w = 16 h4 + kq) hit 32 distinct
+        // banks, the loads (16 consecutive n, two w) at most two per bank.
+        // tbuf word w holds the codes of k = 4w .. 4w+3.
+        auto tcol = [](int n, int w) { return (w + 2 * (n >> 3)) & 31; };
 #pragma unroll
         for (int h4 = 0; h4 < 2; ++h4) {
             Raw8<T> raw[4];
@@ -266,8 +334,8 @@ __global__ void __launch_bounds__(kQsThreads, 1)
                 transpose4x4_bytes(codes[0].y, codes[1].y, codes[2].y, codes[3].y, wy);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    tb[c * 8 + e][h4 * 16 + kq] = wx[e];
-                    tb[c * 8 + 4 + e][h4 * 16 + kq] = wy[e];
+                    tb[c * 8 + e][tcol(c * 8 + e, h4 * 16 + kq)] = wx[e];
+                    tb[c * 8 + 4 + e][tcol(c * 8 + 4 + e, h4 * 16 + kq)] = wy[e];
                 }
             }
         }
@@ -276,19 +344,24 @@ __global__ void __launch_bounds__(kQsThreads, 1)
             if (!group_sync(&tail->gbar[g], gbar_uses, lane, abort_flag)) break;
             const int n = t >> 1;
             const int part = t & 1;
-            uint8_t* dst = p.q + (bc * 128 + n) * p.ldq + br * 128 + part * 64;
+            // Row n of the output block: 128 codes, written as 16-byte
+            // pieces 32 j + 16 part, so that the two lanes of a row fill
+            // whole 32-byte sectors in each store.
+            uint8_t* dst = p.q + (bc * 128 + n) * p.ldq + br * 128 + part * 16;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 uint4 o;
-                o.x = tb[n][part * 16 + j * 4 + 0];
-                o.y = tb[n][part * 16 + j * 4 + 1];
-                o.z = tb[n][part * 16 + j * 4 + 2];
-                o.w = tb[n][part * 16 + j * 4 + 3];
-                __stcs(reinterpret_cast<uint4*>(dst) + j, o);
+                o.x = tb[n][tcol(n, j * 8 + part * 4 + 0)];
+                o.y = tb[n][tcol(n, j * 8 + part * 4 + 1)];
+                o.z = tb[n][tcol(n, j * 8 + part * 4 + 2)];
+                o.w = tb[n][tcol(n, j * 8 + part * 4 + 3)];
+                __stcs(reinterpret_cast<uint4*>(dst + j * 32), o);
             }
-            // tbuf is rewritten for the next box
-            if (!group_sync(&tail->gbar[g], gbar_uses, lane, abort_flag)) break;
+            // No barrier here: this parity of tbuf is written again two boxes
+            // on, after group barriers that every thread reaches only once
+            // its loads above are done.
         }
+        }  // weight modes
     }
     // After an abandoned wait a refill may still be in flight: let it land
     // before the CTA leaves (every fill is consumed on the normal path).
