@@ -92,6 +92,14 @@ struct GemmParams {
     int G;
 };
 
+// Grouped GEMM: the persistent tile schedule, built in shared memory from
+// the device-side offsets at kernel start.
+struct GroupTables {
+    int grp_prefix[kMaxGroups + 1];  // tiles before group g
+    int grp_lo[kMaxGroups];          // first row of group g
+    int grp_hi[kMaxGroups];          // one past its last row (clamped to M)
+};
+
 // Shared-memory layout after the 1024-aligned operand ring.
 struct GemmSmemTail {
     uint64_t full[kStages];
@@ -102,9 +110,7 @@ struct GemmSmemTail {
     int abort_flag;
     int total_tiles;
     int pad;
-    int grp_prefix[kMaxGroups + 1];  // grouped: tiles before group g
-    int grp_lo[kMaxGroups];          // grouped: first row of group g
-    int grp_hi[kMaxGroups];          // grouped: one past its last row (clamped)
+    GroupTables grp;
 };
 
 constexpr size_t kGemmSmemBytes = 1024 /* alignment slack */ + kStages * kStageBytes +
@@ -158,11 +164,49 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     }
 }
 
+// One warp builds the grouped tile table from the device offsets: group g
+// has ceil(rows_g / kTileM) m-tiles times num_nt n-tiles.  Invalid offsets
+// (negative, or decreasing) give an empty group and record FP8_ERR_SHAPE.
+template <int kTileM>
+__device__ __forceinline__ void build_group_tables(const GemmParams& p, GroupTables* gt, int lane,
+                                                   int* total_tiles) {
+    int carry = 0;
+    for (int base = 0; base < p.G; base += 32) {
+        const int g = base + lane;
+        int tiles = 0;
+        if (g < p.G) {
+            int64_t lo = p.offsets[g];
+            int64_t hi = p.offsets[g + 1];
+            if (lo < 0 || hi < lo) {
+                record_device_error(kDevErrShape);
+                lo = hi = 0;
+            }
+            lo = lo < p.M ? lo : p.M;
+            hi = hi < p.M ? hi : p.M;
+            gt->grp_lo[g] = static_cast<int>(lo);
+            gt->grp_hi[g] = static_cast<int>(hi);
+            tiles = static_cast<int>((hi - lo + kTileM - 1) / kTileM) * p.num_nt;
+        }
+        int incl = tiles;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        if (g < p.G) gt->grp_prefix[g + 1] = carry + incl;
+        carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+    if (lane == 0) {
+        gt->grp_prefix[0] = 0;
+        *total_tiles = carry;
+    }
+}
+
 // Tile t of the persistent schedule.  Dense tiles are kTileM rows high;
 // grouped tiles are kBM rows of one group.
 template <bool kGrouped, int kTileM = kBM>
 __device__ __forceinline__ TileCoord decode_tile(int t, const GemmParams& p,
-                                                 const GemmSmemTail* tail) {
+                                                 const GroupTables* gt) {
     TileCoord tc;
     if (!kGrouped) {
         // Bands of band_m m-tiles; inside a band, m runs fastest so that the
@@ -183,16 +227,16 @@ __device__ __forceinline__ TileCoord decode_tile(int t, const GemmParams& p,
         int lo = 0, hi = p.G;  // find the last g with grp_prefix[g] <= t
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
-            if (tail->grp_prefix[mid] <= t) lo = mid; else hi = mid;
+            if (gt->grp_prefix[mid] <= t) lo = mid; else hi = mid;
         }
         const int g = lo;
-        const int local = t - tail->grp_prefix[g];
-        const int rows = tail->grp_hi[g] - tail->grp_lo[g];
-        const int nmt = (rows + kBM - 1) / kBM;
+        const int local = t - gt->grp_prefix[g];
+        const int rows = gt->grp_hi[g] - gt->grp_lo[g];
+        const int nmt = (rows + kTileM - 1) / kTileM;
         const int nt = local / nmt;
         const int mt = local - nt * nmt;  // m fastest: neighbours share B tiles
-        tc.m0 = tail->grp_lo[g] + static_cast<int64_t>(mt) * kBM;
-        tc.row_end = tail->grp_hi[g];
+        tc.m0 = gt->grp_lo[g] + static_cast<int64_t>(mt) * kTileM;
+        tc.row_end = gt->grp_hi[g];
         tc.n0 = static_cast<int64_t>(nt) * kBN;
         tc.g = g;
     }
@@ -333,38 +377,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_relinquish();
     }
     if (kGrouped && warp == kSchedWarp) {
-        // Tile table from the device offsets: group g has ceil(rows_g/128)
-        // m-tiles times num_nt n-tiles.  Invalid offsets give empty groups.
-        int carry = 0;
-        for (int base = 0; base < p.G; base += 32) {
-            const int g = base + lane;
-            int tiles = 0;
-            if (g < p.G) {
-                int64_t lo = p.offsets[g];
-                int64_t hi = p.offsets[g + 1];
-                if (lo < 0 || hi < lo) {
-                    record_device_error(kDevErrShape);
-                    lo = hi = 0;
-                }
-                lo = lo < p.M ? lo : p.M;
-                hi = hi < p.M ? hi : p.M;
-                tail->grp_lo[g] = static_cast<int>(lo);
-                tail->grp_hi[g] = static_cast<int>(hi);
-                tiles = static_cast<int>((hi - lo + kBM - 1) / kBM) * p.num_nt;
-            }
-            int incl = tiles;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-                if (lane >= off) incl += y;
-            }
-            if (g < p.G) tail->grp_prefix[g + 1] = carry + incl;
-            carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
-        }
-        if (lane == 0) {
-            tail->grp_prefix[0] = 0;
-            tail->total_tiles = carry;
-        }
+        build_group_tables<kBM>(p, &tail->grp, lane, &tail->total_tiles);
     } else if (!kGrouped && warp == kSchedWarp && lane == 0) {
         tail->total_tiles = p.num_mt * p.num_nt;
     }
@@ -386,7 +399,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint32_t issued_mask = 0, last_parity = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-                const TileCoord tc = decode_tile<kGrouped>(t, p, tail);
+                const TileCoord tc = decode_tile<kGrouped>(t, p, &tail->grp);
                 const int32_t a_row = static_cast<int32_t>(tc.m0);
                 const int32_t b_row = static_cast<int32_t>(tc.g * p.N + tc.n0);
                 for (int kb = 0; kb < nkb; ++kb) {
@@ -458,7 +471,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint32_t chunk = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-            const TileCoord tc = decode_tile<kGrouped>(t, p, tail);
+            const TileCoord tc = decode_tile<kGrouped>(t, p, &tail->grp);
             const int64_t row = tc.m0 + r;
             const bool row_ok = row < tc.row_end;
             const int64_t col0 = tc.n0 + h * 128;

@@ -1,5 +1,6 @@
-// gemm_pair_kernels.cuh -- dense block-scaled FP8 GEMM on a CTA pair
-// (tcgen05 cta_group::2): one 256 x 256 output tile per pair of SMs.
+// gemm_pair_kernels.cuh -- block-scaled FP8 GEMM on a CTA pair (tcgen05
+// cta_group::2): one 256 x 256 output tile per pair of SMs.  Dense, or
+// grouped (MoE experts: tiles of 256 rows of one group, B and sb per group).
 //
 // Same arithmetic as blockscaled_gemm_kernel (each 128-wide K chunk's
 // tensor-core partial is scaled by sa * sb and added into FP32 registers;
@@ -48,6 +49,8 @@ struct GemmPairSmemTail {
 
 constexpr size_t kGemmPairSmemBytes =
     1024 /* alignment slack */ + kPairStages * kPairStageBytes + sizeof(GemmPairSmemTail);
+// The grouped form adds its tile table (GroupTables) after the tail.
+constexpr size_t kGemmPairGroupedSmemBytes = kGemmPairSmemBytes + sizeof(GroupTables);
 
 __device__ __forceinline__ void spin_ns(uint64_t ns) {
     const uint64_t t0 = globaltimer_ns();
@@ -55,7 +58,7 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
     }
 }
 
-template <bool kOutBf16>
+template <bool kGrouped, bool kOutBf16>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     blockscaled_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                                  const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
@@ -64,6 +67,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
     GemmPairSmemTail* tail =
         reinterpret_cast<GemmPairSmemTail*>(smem + kPairStages * kPairStageBytes);
+    GroupTables* gt = reinterpret_cast<GroupTables*>(tail + 1);   // grouped only
     volatile int* abort_flag = &tail->abort_flag;
     auto stage_a = [&](int s) { return smem + s * kPairStageBytes; };
     auto stage_b = [&](int s) { return smem + s * kPairStageBytes + kPairHalfBytes; };
@@ -85,7 +89,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(&tail->tempty[b], 2 * kEpiWarps);
         }
         tail->abort_flag = 0;
-        tail->total_tiles = p.num_mt * p.num_nt;
+        if (!kGrouped) tail->total_tiles = p.num_mt * p.num_nt;
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
@@ -94,6 +98,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_alloc_pair(&tail->tmem_base, kTmemCols);
         tmem_relinquish_pair();
     }
+    if (kGrouped && warp == kSchedWarp)   // both CTAs build the same table
+        build_group_tables<kPairBM>(p, gt, lane, &tail->total_tiles);
     tc_fence_before();
     cluster_sync();
     tc_fence_after();
@@ -112,9 +118,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint32_t used_mask = 0, last_parity = 0;
             bool ok = true;
             for (int t = pair; t < total_tiles && ok; t += num_pairs) {
-                const TileCoord tc = decode_tile<false, kPairBM>(t, p, nullptr);
+                const TileCoord tc = decode_tile<kGrouped, kPairBM>(t, p, gt);
                 const int32_t a_row = static_cast<int32_t>(tc.m0) + 128 * static_cast<int32_t>(rank);
-                const int32_t b_row = static_cast<int32_t>(tc.n0) + 128 * static_cast<int32_t>(rank);
+                // grouped: expert g's weights are rows [g N, g N + N) of B
+                const int32_t b_row = static_cast<int32_t>(static_cast<int64_t>(tc.g) * p.N + tc.n0) +
+                                      128 * static_cast<int32_t>(rank);
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!bounded_wait(&tail->empty[stage], phase ^ 1u, abort_flag)) {
                         ok = false;
@@ -210,14 +218,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint32_t chunk = 0;
         bool ok = true;
         for (int t = pair; t < total_tiles && ok; t += num_pairs) {
-            const TileCoord tc = decode_tile<false, kPairBM>(t, p, nullptr);
+            const TileCoord tc = decode_tile<kGrouped, kPairBM>(t, p, gt);
             const int64_t row = tc.m0 + r;
             const bool row_ok = row < tc.row_end;
             const int64_t col0 = tc.n0 + h * 128;
             const bool col_ok = col0 < p.N;
             ok = epilogue_tile<kOutBf16>(
                 p, tail->tfull, abort_flag, tmem_base, t_lane, h, lane, row, row_ok, col0, col_ok,
-                0, chunk, [&](uint32_t buf) { mbar_arrive_cluster(tempty_leader[buf]); });
+                tc.g, chunk, [&](uint32_t buf) { mbar_arrive_cluster(tempty_leader[buf]); });
         }
         if (!ok) aborted = true;
     }
