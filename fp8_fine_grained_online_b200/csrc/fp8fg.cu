@@ -16,7 +16,6 @@
 #include "gemm_pair_kernels.cuh"
 #include "quant_kernels.cuh"
 #include "quant_stream_kernels.cuh"
-#include "quant_act_kernels.cuh"
 
 namespace fp8fg {
 namespace {
@@ -181,9 +180,6 @@ inline fp8_status_t launch_status() {
 // faster on one CTA).
 constexpr int64_t kGroupedPairMinK = 4096;
 
-// Activation quantization: TMA-streamed boxes (true) or register tiles (false).
-constexpr bool kActUseStream = true;
-
 int elem_size_in(fp8_in_t t) { return t == FP8_IN_BF16 ? 2 : (t == FP8_IN_FP32 ? 4 : 0); }
 int elem_size_out(fp8_out_t t) { return t == FP8_OUT_BF16 ? 2 : (t == FP8_OUT_FP32 ? 4 : 0); }
 
@@ -328,38 +324,12 @@ fp8_status_t fp8_quantize_act_1x128(const void* x, fp8_in_t x_type, int64_t M, i
     int dev, sms;
     fp8_status_t st = current_device(&dev, &sms);
     if (st != FP8_OK) return st;
-    if (kActUseStream) {
-        QsParams p{};
-        p.rows = M; p.cols = K;
-        p.nbr = (M + 127) / 128; p.nbc = K / 128;
-        p.q = q; p.ldq = ldq;
-        p.s = sa; p.s_stride_r = sa_stride_m; p.s_stride_c = sa_stride_kb;
-        return launch_quant_stream(x, x_type, ldx, p, kQuantAct, sms, stream);
-    }
-    const int64_t nkb = K / 128;
-    const int64_t tiles = M * nkb;
-    const int64_t grid = grid_for((tiles + kActTilesPerStep - 1) / kActTilesPerStep, sms, kActMinBlocks);
-    const bool small = tiles + grid * kActTilesPerStep < (static_cast<int64_t>(1) << 31);
-    const FastDivU31 fd = FastDivU31::make(small ? static_cast<uint32_t>(nkb) : 1u);
-    const unsigned g = static_cast<unsigned>(grid);
-    if (x_type == FP8_IN_BF16) {
-        const uint16_t* xs = static_cast<const uint16_t*>(x);
-        if (small)
-            quant_act_1x128_kernel<uint16_t, true><<<g, kActThreads, 0, stream>>>(
-                xs, M, nkb, fd, ldx, q, ldq, sa, sa_stride_m, sa_stride_kb);
-        else
-            quant_act_1x128_kernel<uint16_t, false><<<g, kActThreads, 0, stream>>>(
-                xs, M, nkb, fd, ldx, q, ldq, sa, sa_stride_m, sa_stride_kb);
-    } else {
-        const float* xs = static_cast<const float*>(x);
-        if (small)
-            quant_act_1x128_kernel<float, true><<<g, kActThreads, 0, stream>>>(
-                xs, M, nkb, fd, ldx, q, ldq, sa, sa_stride_m, sa_stride_kb);
-        else
-            quant_act_1x128_kernel<float, false><<<g, kActThreads, 0, stream>>>(
-                xs, M, nkb, fd, ldx, q, ldq, sa, sa_stride_m, sa_stride_kb);
-    }
-    return launch_status();
+    QsParams p{};
+    p.rows = M; p.cols = K;
+    p.nbr = (M + 127) / 128; p.nbc = K / 128;
+    p.q = q; p.ldq = ldq;
+    p.s = sa; p.s_stride_r = sa_stride_m; p.s_stride_c = sa_stride_kb;
+    return launch_quant_stream(x, x_type, ldx, p, kQuantAct, sms, stream);
 }
 
 fp8_status_t fp8_quantize_weight_128x128(const void* w, fp8_in_t w_type, int64_t K, int64_t N,

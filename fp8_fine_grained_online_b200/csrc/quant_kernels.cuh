@@ -275,28 +275,6 @@ __device__ __forceinline__ void patch_pair(uint2& codes, int k, uint32_t c16) {
         codes.y = (codes.y & keep) | (c16 << sh);
 }
 
-// floor(n / d) for 0 <= n < 2^31 and a fixed d >= 1, by multiplication:
-// with l = ceil(log2 d) and m = ceil(2^(31+l) / d), 2^(31+l) <= m d <=
-// 2^(31+l) + 2^l, so floor(n / d) = (n m) >> (31 + l) (Granlund and
-// Montgomery, "Division by invariant integers using multiplication", 1994,
-// round-up method).  m <= 2^32 keeps n m below 2^63.
-struct FastDivU31 {
-    uint64_t m;
-    int shift;
-    __host__ static FastDivU31 make(uint32_t d) {  // d < 2^31
-        int l = 0;
-        while ((static_cast<uint64_t>(1) << l) < d) ++l;
-        FastDivU31 f;
-        const uint64_t num = static_cast<uint64_t>(1) << (31 + l);  // l <= 31
-        f.m = (num + d - 1) / d;
-        f.shift = 31 + l;
-        return f;
-    }
-    __device__ __forceinline__ uint32_t div(uint32_t n) const {
-        return static_cast<uint32_t>((static_cast<uint64_t>(n) * m) >> shift);
-    }
-};
-
 // C = 0 for a GEMM with an empty contraction (K == 0).
 template <typename T>
 __global__ void __launch_bounds__(256)
