@@ -79,21 +79,23 @@ fp8_status_t current_device(int* dev_out, int* sms_out) {
                         return FP8_ERR_CUDA;
                     }
                 }
-                const void* qs_bf16[] = {
+                const void* qs_kernels[] = {
                     reinterpret_cast<const void*>(&quant_stream_kernel<uint16_t, kQuantAct>),
                     reinterpret_cast<const void*>(&quant_stream_kernel<uint16_t, kQuantWeight>),
-                    reinterpret_cast<const void*>(&quant_stream_kernel<uint16_t, kQuantWeightT>)};
-                const void* qs_f32[] = {
+                    reinterpret_cast<const void*>(&quant_stream_kernel<uint16_t, kQuantWeightT>),
                     reinterpret_cast<const void*>(&quant_stream_kernel<float, kQuantAct>),
                     reinterpret_cast<const void*>(&quant_stream_kernel<float, kQuantWeight>),
                     reinterpret_cast<const void*>(&quant_stream_kernel<float, kQuantWeightT>)};
-                for (int i = 0; i < 3; ++i) {
-                    if (cudaFuncSetAttribute(qs_bf16[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(quant_stream_smem_bytes<uint16_t>())) !=
-                            cudaSuccess ||
-                        cudaFuncSetAttribute(qs_f32[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(quant_stream_smem_bytes<float>())) !=
-                            cudaSuccess) {
+                const size_t qs_bytes[] = {quant_stream_smem_bytes<uint16_t, kQuantAct>(),
+                                           quant_stream_smem_bytes<uint16_t, kQuantWeight>(),
+                                           quant_stream_smem_bytes<uint16_t, kQuantWeightT>(),
+                                           quant_stream_smem_bytes<float, kQuantAct>(),
+                                           quant_stream_smem_bytes<float, kQuantWeight>(),
+                                           quant_stream_smem_bytes<float, kQuantWeightT>()};
+                for (int i = 0; i < 6; ++i) {
+                    if (cudaFuncSetAttribute(qs_kernels[i],
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(qs_bytes[i])) != cudaSuccess) {
                         cudaGetLastError();
                         return FP8_ERR_CUDA;
                     }
@@ -234,8 +236,12 @@ fp8_status_t launch_quant_stream_t(const CUtensorMap& map, const QsParams& p, in
                                    cudaStream_t stream) {
     const int64_t boxes = p.nbr * p.nbc;
     const unsigned grid = static_cast<unsigned>(boxes < sms ? boxes : sms);
+    QsParams q = p;
+    const int64_t step = static_cast<int64_t>(kQsGroups) * grid;
+    q.step_r = step / p.nbc;
+    q.step_c = step - q.step_r * p.nbc;
     quant_stream_kernel<T, kMode>
-        <<<grid, kQsThreads, quant_stream_smem_bytes<T>(), stream>>>(map, p);
+        <<<grid, kQsThreads, quant_stream_smem_bytes<T, kMode>(), stream>>>(map, q);
     return launch_status();
 }
 

@@ -40,14 +40,14 @@ struct Raw8<uint16_t> {  // bf16 bit patterns
             v[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
         }
     }
-    // The 8 elements negated (one IMAD / LOP3 each, like to_float).
-    __device__ __forceinline__ void to_neg_float(float (&v)[8]) const {
+    // The 8 elements negated, as 4 packed fp32 pairs (one IMAD / LOP3 per
+    // element, like to_float).
+    __device__ __forceinline__ void to_neg_pairs(uint64_t (&v)[4]) const {
         const uint32_t u[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            v[2 * i] = __uint_as_float((u[i] << 16) ^ 0x80000000u);
-            v[2 * i + 1] = __uint_as_float((u[i] & 0xFFFF0000u) ^ 0x80000000u);
-        }
+        for (int i = 0; i < 4; ++i)
+            v[i] = f2_pack(__uint_as_float((u[i] << 16) ^ 0x80000000u),
+                           __uint_as_float((u[i] & 0xFFFF0000u) ^ 0x80000000u));
     }
     // max |x| of the 8 elements (exact; NaN elements are skipped), on packed
     // bf16 pairs: clear the sign bits, then lane-wise maxima.
@@ -148,18 +148,6 @@ __device__ __forceinline__ bool reciprocal_path_ok(float s) {
     return s >= 0x1p-125f && s <= 0x1p125f;
 }
 
-// (a0, a1) * (b0, b1), each lane IEEE round-to-nearest (packed sm_100 FMUL).
-__device__ __forceinline__ void fmul2(float& d0, float& d1, float a0, float a1, float b0,
-                                      float b1) {
-    asm("{\n\t.reg .b64 ta, tb, td;\n\t"
-        "mov.b64 ta, {%2, %3};\n\t"
-        "mov.b64 tb, {%4, %5};\n\t"
-        "mul.rn.f32x2 td, ta, tb;\n\t"
-        "mov.b64 {%0, %1}, td;\n\t}"
-        : "=f"(d0), "=f"(d1)
-        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-
 // Bracket-path codes of 8 values, branch free.  Bit k of the returned
 // `amb` is set when the bracket ends disagree for elements 2k or 2k+1 (the
 // quotient lies within ~2^-20 of an E4M3 rounding midpoint).  For bf16 data
@@ -172,9 +160,10 @@ __device__ __forceinline__ uint2 encode8_bracket(const float (&v)[8], float ru, 
     amb = 0;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
+        const uint64_t x2 = f2_pack(v[2 * k], v[2 * k + 1]);
         float u0, u1, d0, d1;
-        fmul2(u0, u1, v[2 * k], v[2 * k + 1], ru, ru);
-        fmul2(d0, d1, v[2 * k], v[2 * k + 1], rd, rd);
+        f2_unpack(f2_mul(x2, f2_pack(ru, ru)), u0, u1);
+        f2_unpack(f2_mul(x2, f2_pack(rd, rd)), d0, d1);
         hi[k] = cvt_e4m3x2(u0, u1);
         amb |= (hi[k] != cvt_e4m3x2(d0, d1) ? 1u : 0u) << k;
     }
@@ -206,17 +195,19 @@ __device__ __forceinline__ bool corrected_path_ok(float s) {
     return s >= 0x1p-100f && s <= 0x1p125f;
 }
 
-// n: the 8 inputs negated; neg_r = -RN32(1 / s).
-__device__ __forceinline__ uint2 encode8_corrected(const float (&n)[8], float s, float neg_r) {
+// n: the 8 inputs negated, as 4 packed pairs; s2 = (s, s); neg_r2 = (-r, -r)
+// with r = RN32(1 / s).
+__device__ __forceinline__ uint2 encode8_corrected(const uint64_t (&n)[4], uint64_t s2,
+                                                   uint64_t neg_r2) {
     uint32_t c[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        float q0, q1;
-        fmul2(q0, q1, n[2 * k], n[2 * k + 1], neg_r, neg_r);
-        float t0 = n[2 * k], t1 = n[2 * k + 1];
-        ffma2_scalar(t0, t1, s, q0, q1);          // q0 s - x, exact
-        ffma2_scalar(q0, q1, neg_r, t0, t1);      // q0 - t r
-        c[k] = cvt_e4m3x2(q0, q1);
+        const uint64_t q0 = f2_mul(n[k], neg_r2);           // x r
+        const uint64_t t = f2_fma(q0, s2, n[k]);             // q0 s - x, exact
+        const uint64_t q1 = f2_fma(t, neg_r2, q0);           // q0 - t r
+        float lo, hi;
+        f2_unpack(q1, lo, hi);
+        c[k] = cvt_e4m3x2(lo, hi);
     }
     uint2 out;
     out.x = c[0] | (c[1] << 16);

@@ -35,25 +35,37 @@ enum QuantMode { kQuantAct = 0, kQuantWeight = 1, kQuantWeightT = 2 };
 constexpr int kQsGroups = 2;                 // consumer groups of 8 warps
 constexpr int kQsThreads = kQsGroups * 256;
 
-template <typename T>
+constexpr int kQsMaxStages = 4;
+
+// Ring per group: two 32 KB bf16 boxes or one 64 KB fp32 box.  (Three bf16
+// boxes per group measured no faster for activations and slower for [K,N]
+// weights.)
+template <typename T, int kMode>
 struct QsCfg {
-    static constexpr int kSlots = sizeof(T) == 2 ? 2 : 1;   // ring slots per group
+    static constexpr bool kTransposed = kMode == kQuantWeightT;
+    static constexpr int kSlots = sizeof(T) == 2 ? 2 : 1;
     static constexpr int kStages = kQsGroups * kSlots;
     static constexpr int kBoxBytes = 128 * 128 * static_cast<int>(sizeof(T));
     static constexpr int kRowBytes = 128 * static_cast<int>(sizeof(T));
+    static_assert(kStages <= kQsMaxStages, "ring too long");
 };
 
 struct QsSmemTail {
-    uint64_t full[4];                  // slot filled (TMA bytes)
+    uint64_t full[kQsMaxStages];       // slot filled (TMA bytes)
     uint64_t gbar[kQsGroups];          // per-group barrier (8 warp arrivals)
     float red[kQsGroups][2][8];        // [group][block parity][warp]
-    uint32_t tbuf[kQsGroups][2][128][33]; // [group][box parity][n][k/4 swizzled], transposed codes
     int abort_flag;
 };
 
-template <typename T>
+// [N, K] output only: [group][box parity][n][k/4 swizzled], transposed codes.
+struct QsTransposeBuf {
+    uint32_t tbuf[kQsGroups][2][128][33];
+};
+
+template <typename T, int kMode>
 constexpr size_t quant_stream_smem_bytes() {
-    return 1024 + QsCfg<T>::kStages * QsCfg<T>::kBoxBytes + sizeof(QsSmemTail);
+    return 1024 + QsCfg<T, kMode>::kStages * QsCfg<T, kMode>::kBoxBytes + sizeof(QsSmemTail) +
+           (QsCfg<T, kMode>::kTransposed ? sizeof(QsTransposeBuf) : 0);
 }
 
 struct QsParams {
@@ -63,6 +75,26 @@ struct QsParams {
     int64_t ldq;
     float* s;
     int64_t s_stride_r, s_stride_c;   // act: (m, kb); weight: (kb, nb)
+    // A group's consecutive boxes are kQsGroups * gridDim.x apart: that
+    // step as (box rows, box columns) with step_c < nbc, set by the host.
+    int64_t step_r, step_c;
+};
+
+// (box row, box column) of a group's box sequence, advanced without dividing.
+struct BoxCursor {
+    int64_t br, bc;
+    __device__ __forceinline__ void init(int64_t box, int64_t nbc) {
+        br = box / nbc;
+        bc = box - br * nbc;
+    }
+    __device__ __forceinline__ void advance(const QsParams& p) {
+        bc += p.step_c;
+        br += p.step_r;
+        if (bc >= p.nbc) {
+            bc -= p.nbc;
+            ++br;
+        }
+    }
 };
 
 // Barrier of one consumer group (its 8 warps) through an mbarrier, so that
@@ -122,12 +154,14 @@ __device__ __forceinline__ void transpose4x4_bytes(uint32_t r0, uint32_t r1, uin
 template <typename T, int kMode>
 __global__ void __launch_bounds__(kQsThreads, 1)
     quant_stream_kernel(const __grid_constant__ CUtensorMap tm_in, const QsParams p) {
-    constexpr int kSlots = QsCfg<T>::kSlots;
-    constexpr int kStages = QsCfg<T>::kStages;
-    constexpr int kBoxBytes = QsCfg<T>::kBoxBytes;
+    using Cfg = QsCfg<T, kMode>;
+    constexpr int kSlots = Cfg::kSlots;
+    constexpr int kStages = Cfg::kStages;
+    constexpr int kBoxBytes = Cfg::kBoxBytes;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     QsSmemTail* tail = reinterpret_cast<QsSmemTail*>(smem + kStages * kBoxBytes);
+    QsTransposeBuf* tx = reinterpret_cast<QsTransposeBuf*>(tail + 1);   // [N, K] output only
     volatile int* abort_flag = &tail->abort_flag;
 
     const int warp = threadIdx.x >> 5;
@@ -159,14 +193,17 @@ __global__ void __launch_bounds__(kQsThreads, 1)
     // a slot is refilled once the whole group has read it.
     auto box_of = [&](int64_t k) { return g + kQsGroups * k; };
     auto slot_of = [&](int64_t k) { return g * kSlots + static_cast<int>(k % kSlots); };
+    // Boxes are issued in order k = 0, 1, ... (by the group's thread 0) and
+    // consumed in the same order: one cursor each.
+    BoxCursor issue_at, box_at;
+    issue_at.init(blockIdx.x + static_cast<int64_t>(g) * gridDim.x, p.nbc);
+    box_at = issue_at;
     auto issue = [&](int64_t k) {
-        const int64_t box = blockIdx.x + box_of(k) * gridDim.x;
-        const int64_t br = box / p.nbc;
-        const int64_t bc = box - br * p.nbc;
         const int slot = slot_of(k);
         mbar_arrive_expect_tx(&tail->full[slot], kBoxBytes);
         tma_load_2d(smem + slot * kBoxBytes, &tm_in, &tail->full[slot],
-                    static_cast<int32_t>(bc * 128), static_cast<int32_t>(br * 128));
+                    static_cast<int32_t>(issue_at.bc * 128), static_cast<int32_t>(issue_at.br * 128));
+        issue_at.advance(p);
     };
     if (t == 0)
         for (int64_t k = 0; k < kSlots && box_of(k) < count; ++k) issue(k);
@@ -177,7 +214,7 @@ __global__ void __launch_bounds__(kQsThreads, 1)
         const uint32_t phase = static_cast<uint32_t>((k / kSlots) & 1);
         if (!bounded_wait(&tail->full[stage], phase, abort_flag)) break;
         const uint8_t* box_smem = smem + stage * kBoxBytes;
-        auto row_ptr = [&](int j) { return box_smem + row_in_box(j) * QsCfg<T>::kRowBytes; };
+        auto row_ptr = [&](int j) { return box_smem + row_in_box(j) * Cfg::kRowBytes; };
         // The group has finished reading the slot: refill it with the
         // group's box k + kSlots.
         auto release_stage = [&]() -> bool {
@@ -185,9 +222,9 @@ __global__ void __launch_bounds__(kQsThreads, 1)
             if (t == 0 && box_of(k + kSlots) < count) issue(k + kSlots);
             return true;
         };
-        const int64_t box = blockIdx.x + i * gridDim.x;
-        const int64_t br = box / p.nbc;
-        const int64_t bc = box - br * p.nbc;
+        const int64_t br = box_at.br;
+        const int64_t bc = box_at.bc;
+        box_at.advance(p);
 
         if constexpr (kMode == kQuantAct) {
             // One 1x128 tile per row: the 16 lanes of a half-warp share 8
@@ -219,9 +256,9 @@ __global__ void __launch_bounds__(kQsThreads, 1)
                 uint2 codes;
                 if constexpr (sizeof(T) == 2) {
                     const float neg_r = __shfl_sync(0xFFFFFFFFu, -my_r, half_base + j);
-                    float n[8];
-                    raw[j].to_neg_float(n);
-                    codes = encode8_corrected(n, sj[j], neg_r);
+                    uint64_t n[4];
+                    raw[j].to_neg_pairs(n);
+                    codes = encode8_corrected(n, f2_pack(sj[j], sj[j]), f2_pack(neg_r, neg_r));
                     amb4 = corrected_path_ok(sj[j]) ? 0u : 0xFu;
                 } else {
                     const float ru = __shfl_sync(0xFFFFFFFFu, my_r * kBracketUp, half_base + j);
@@ -275,8 +312,10 @@ __global__ void __launch_bounds__(kQsThreads, 1)
         const float ru = rcp * kBracketUp;
         const float rd = rcp * kBracketDown;
         const bool off_path = sizeof(T) == 2 ? !corrected_path_ok(s) : !reciprocal_path_ok(s);
+        const uint64_t s2 = f2_pack(s, s);
+        const uint64_t neg_r2 = f2_pack(-rcp, -rcp);
         if (t == 0) p.s[br * p.s_stride_r + bc * p.s_stride_c] = s;
-        uint32_t(*tb)[33] = tail->tbuf[g][par];
+        uint32_t(*tb)[33] = tx->tbuf[g][par];
         // Word w of row n sits at column (w + 2 (n / 8)) mod 32 of a 33-word
         // row: the stores below (n = 8c + e, w = 16 h4 + kq) hit 32 distinct
         // banks, the loads (16 consecutive n, two w) at most two per bank.
@@ -297,9 +336,9 @@ __global__ void __launch_bounds__(kQsThreads, 1)
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
                 if constexpr (sizeof(T) == 2) {
-                    float n[8];
-                    raw[jj].to_neg_float(n);
-                    codes[jj] = encode8_corrected(n, s, -rcp);
+                    uint64_t n[4];
+                    raw[jj].to_neg_pairs(n);
+                    codes[jj] = encode8_corrected(n, s2, neg_r2);
                 } else {
                     float v[8];
                     raw[jj].to_float(v);

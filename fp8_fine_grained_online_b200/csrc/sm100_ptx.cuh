@@ -245,6 +245,34 @@ __device__ __forceinline__ void tmem_wait_ld_dep(uint32_t (&r)[32]) {
         : "memory");
 }
 
+// Two fp32 values in one 64-bit register pair (lo in the low half), and the
+// packed sm_100 FP32 operations on such pairs (each lane IEEE round-to-
+// nearest, subnormals kept).  Values stay in 64-bit registers from one
+// operation to the next.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+// a * b
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// a * b + c
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 // Packed FP32 FMA on sm_100: (d0, d1) = s * (b0, b1) + (d0, d1), each lane
 // rounded to nearest even like fmaf.
 __device__ __forceinline__ void ffma2_scalar(float& d0, float& d1, float s, float b0, float b1) {
