@@ -10,17 +10,19 @@
 // tensor-core partial sums are promoted to FP32 registers at fixed
 // intervals; "Finkornig kvantisering" for the 1x128 / 128x128 scales).
 //
-// Structure (one persistent CTA per SM, 320 threads):
-//   warp 0      TMA producer: A tile 128x128 B and B tile 256x128 B per chunk
+// Structure of the one-CTA kernel (one persistent CTA per SM, 384 threads;
+// the CTA-pair kernel in gemm_pair_kernels.cuh has the same roles):
+//   warps 0-7   epilogue: warp w reads TMEM lanes 32*(w%4).. and columns
+//               128*(w/4).., scales the chunk partial by sa*sb and adds it
+//               to 128 FP32 accumulators per thread (one output row, 128
+//               columns); at tile end converts and stores the row.
+//   warp 8      TMA producer: A tile 128x128 B and B tile 256x128 B per chunk
 //               into a 4-stage shared-memory ring (128-byte swizzle).
-//   warp 1      TMEM owner and MMA issuer: per chunk, 4 x UMMA
+//   warp 9      TMEM owner and MMA issuer: per chunk, 4 x UMMA
 //               (M=128, N=256, K=32) into one of two TMEM partial buffers
 //               (2 x 256 columns), then commits to the ring's "empty"
 //               barrier and the buffer's "full" barrier.
-//   warps 2-9   epilogue: warp w reads TMEM lanes 32*(w%4).. and columns
-//               128*((w-2)/4).., scales the chunk partial by sa*sb and adds
-//               it to 128 FP32 accumulators per thread (one output row,
-//               128 columns); at tile end converts and stores the row.
+//   warp 10     grouped: builds the tile table at start; warp 11 idle.
 // Double-buffered TMEM lets the MMA of chunk kb+1 run while the epilogue
 // promotes chunk kb.
 //

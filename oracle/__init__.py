@@ -207,3 +207,24 @@ def dequantize(q, s, tile_rows, tile_cols):
     s64 = np.asarray(s, dtype=np.float64)
     rs = np.repeat(np.repeat(s64, tile_rows, axis=0), tile_cols, axis=1)
     return v * rs[: v.shape[0], : v.shape[1]]
+
+
+def dequantize_fp32(q, s, tile_rows, tile_cols=128):
+    """The dequantized tensor in fp32: E4M3 value of each code times its
+    tile's scale, rounded once to fp32 ([HS] 2.2 dequantize: code value x
+    scale, computed in fp32).  The product of a 4-bit E4M3 significand and a
+    24-bit fp32 scale is exact in fp64, so rounding the fp64 product to fp32
+    is the single correctly rounded fp32 multiply.  Tiles are tile_rows x
+    tile_cols (1 x 128 activations, 128 x 128 weights); NaN codes give NaN."""
+    return dequantize(q, s, tile_rows, tile_cols).astype(np.float32)
+
+
+def f32_to_bf16_bits(x):
+    """bf16 bit patterns of fp32 values, round to nearest, ties to even (the
+    16 high bits after adding 0x7FFF plus the lowest kept bit); NaN stays a
+    quiet NaN."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+    nan = np.isnan(np.asarray(x, dtype=np.float32))
+    r[nan] = ((u[nan] >> 16) | 0x40).astype(np.uint16)
+    return r
