@@ -295,6 +295,67 @@ class Quant(Workload):
         return float(moved)
 
 
+class Dequant(Workload):
+    """Codes back to bf16: the FFN weight W [7168 x 18432] quantized in 128x128
+    blocks (untransposed), dequantized every step."""
+    name = "dequant_w7168x18432_bf16"
+    unit = "GB/s"
+    dominant = "dequantize"
+    sample_text = "%d rows x %d 128-column blocks of the codes, dequantized to bf16"
+
+    def __init__(self, fp8, device, K=7168, N=18432):
+        self.fp8, self.K, self.N = fp8, K, N
+        self.kernels = ["dequantize"]
+        if device is None:
+            return
+        w = synth.weight_input(K, N, 0.02, synth.FFN.config_id, device)
+        self.q, self.s = fp8.fp8_quantize_weight_128x128(w, transpose_out=False)
+        del w
+        self.out = torch.empty((K, N), dtype=torch.bfloat16, device=device)
+
+    def config(self):
+        return {"workload": self.name, "codes": "E4M3 [%dx%d], 128x128 block scales" % (self.K, self.N),
+                "out": "bf16", "source": "FFN W N(0,0.02) quantized once before timing",
+                "l2": "codes 132 MB + output 264 MB > L2"}
+
+    def algorithmic(self):
+        K, N = self.K, self.N
+        return {"dequantize": ("bytes", K * N * 3 + (K // 128) * (N // 128) * 4)}
+
+    def work_per_step(self):
+        return sum(v for _, v in self.algorithmic().values())
+
+    def step(self, marks):
+        marks(0)
+        self.fp8.fp8_dequantize(self.q, self.s, 128, out=self.out)
+        marks(1)
+
+    def e2e_setup(self):
+        self.hq = self.q.cpu().pin_memory()
+        self.hs = self.s.cpu().pin_memory()
+        self.hout = torch.empty((self.K, self.N), dtype=torch.bfloat16, pin_memory=True)
+        return self.hq.numel() + self.hs.numel() * 4, self.hout.numel() * 2
+
+    def e2e_step(self):
+        q = self.hq.to("cuda", non_blocking=True)
+        s = self.hs.to("cuda", non_blocking=True)
+        self.hout.copy_(self.fp8.fp8_dequantize(q, s, 128), non_blocking=True)
+
+    def oracle_sample(self, orc, rows, nbs):
+        # codes of the first nbs column blocks (quantized once, untimed use
+        # of the oracle's quantizer; re-made when a wider sample is asked for)
+        if getattr(self, "_cpu_nbs", 0) < nbs:
+            w = synth.weight_input(self.K, self.N, 0.02, synth.FFN.config_id, "cpu")
+            blk = w[:, :nbs * 128].contiguous().view(torch.int16).numpy().view(np.uint16)
+            self._cpu, self._cpu_nbs = orc.quantize_weight_128x128(blk), nbs
+        q, s = self._cpu
+        n = min(rows * 8, q.shape[0])
+        qs = q[:n, :nbs * 128]
+        out = orc.dequantize_fp32(qs, s[: (n + 127) // 128, :nbs], 128)
+        orc.f32_to_bf16_bits(out)
+        return float(qs.size * 3 + ((n + 127) // 128) * nbs * 4)
+
+
 class DGrad(FFN):
     """dX = dY W^T with W quantized untransposed (K-major for this product)."""
     name = synth.DGRAD.name
@@ -479,11 +540,13 @@ class MoE(Workload):
         return flops
 
 
-WORKLOADS = {"ffn": FFN, "quant": Quant, "moe": MoE, "dgrad": DGrad}
+WORKLOADS = {"ffn": FFN, "quant": Quant, "moe": MoE, "dgrad": DGrad, "dequant": Dequant}
 # Oracle sample per step: (rows, column blocks), sized for a few seconds per step.
-ORACLE_SAMPLE = {"ffn": (32, 2), "quant": (16, 4), "moe": (32, 1), "dgrad": (16, 1)}
-# The single CPU-baseline measurement of the default run: ~10 s of oracle work.
-CPU_BASELINE_SAMPLE = {"ffn": (128, 12), "quant": (64, 24), "moe": (128, 6), "dgrad": (64, 4)}
+ORACLE_SAMPLE = {"ffn": (32, 2), "quant": (16, 4), "moe": (32, 1), "dgrad": (16, 1),
+                 "dequant": (64, 8)}
+# The single CPU-baseline measurement of a run: about 10 s of oracle work.
+CPU_BASELINE_SAMPLE = {"ffn": (512, 36), "quant": (256, 72), "moe": (256, 12), "dgrad": (128, 8),
+                       "dequant": (896, 120)}
 
 
 # ----------------------------------------------------------------------------- timing
@@ -609,14 +672,14 @@ def cpu_baseline(args, wl_cls):
     import oracle
     wl = wl_cls(None, None)
     rows, nbs = CPU_BASELINE_SAMPLE[args.workload]
-    wl.oracle_sample(oracle, 1, 1)              # input generation + library load, untimed
+    wl.oracle_sample(oracle, 1, nbs)            # input generation + library load, untimed
     t0 = time.perf_counter()
     work = wl.oracle_sample(oracle, rows, nbs)
     dt = time.perf_counter() - t0
     return {"value": round(work / dt / scale(wl), 6), "unit": wl.unit,
             "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": "%d rows x %d 128-column blocks of the step, with their online "
-                      "quantization (%.1f s)" % (rows, nbs, dt)}
+            "sample": getattr(wl, "sample_text", "%d rows x %d 128-column blocks of the step, "
+                              "with their online quantization") % (rows, nbs) + " (%.1f s)" % dt}
 
 
 def main():
@@ -645,9 +708,9 @@ def main():
         import oracle
         wl = wl_cls(None, None)
         rows, nbs = ORACLE_SAMPLE[args.workload]
-        wl.oracle_sample(oracle, 1, 1)
+        wl.oracle_sample(oracle, 1, nbs)
         for _ in range(args.warmup):
-            wl.oracle_sample(oracle, 2, 1)
+            wl.oracle_sample(oracle, 2, nbs)
         t0 = time.perf_counter()
         work = 0.0
         for _ in range(args.steps):

@@ -149,6 +149,22 @@ def fp8_grouped_gemm(a, sa, b, sb, offsets, out_dtype=torch.bfloat16, c=None, st
     return c
 
 
+def fp8_dequantize(q, s, tile_rows, out_dtype=torch.bfloat16, out=None, stream=None):
+    """q uint8 [R, C] E4M3 codes with scales s (tile_rows x 128 tiles:
+    tile_rows 1 for activations, s [R, C/128]; 128 for weights,
+    s [R/128, C/128]) -> E4M3(q) * scale as out_dtype [R, C]."""
+    _rowmajor(q, "q")
+    R, C = q.shape
+    if out is None:
+        out = torch.empty((R, C), dtype=out_dtype, device=q.device)
+    _rowmajor(out, "out")
+    st = _L.fp8_dequantize(_ptr(q), R, C, q.stride(0), _ptr(s), s.stride(0), s.stride(1),
+                           tile_rows, _ptr(out), _out_type(out.dtype), out.stride(0),
+                           _stream(stream))
+    _lib.check(st, "fp8_dequantize")
+    return out
+
+
 def linear_forward(x, w, out_dtype=torch.bfloat16, stream=None):
     """Online-quantized FP8 linear layer: y = x @ w with x [M, K], w [K, N].
 

@@ -30,6 +30,8 @@ SIGNATURES = {
                                     _vp, _int, _i64, _i64, _i64, _i64, _vp]),
     "fp8_grouped_gemm": (_int, [_vp, _i64, _vp, _i64, _i64, _vp, _i64, _vp, _i64, _i64, _i64,
                                 _vp, _int, _i64, _vp, _int, _i64, _i64, _i64, _vp]),
+    "fp8_dequantize": (_int, [_vp, _i64, _i64, _i64, _vp, _i64, _i64, _int, _vp, _int, _i64,
+                              _vp]),
     "fp8_status_string": (ctypes.c_char_p, [_int]),
     "fp8_get_device_error": (_int, [_vp, ctypes.POINTER(_int)]),
 }

@@ -16,6 +16,7 @@
 #include "gemm_pair_kernels.cuh"
 #include "quant_kernels.cuh"
 #include "quant_stream_kernels.cuh"
+#include "dequant_kernels.cuh"
 
 namespace fp8fg {
 namespace {
@@ -297,6 +298,36 @@ fp8_status_t launch_pair_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, co
 using namespace fp8fg;
 
 extern "C" {
+
+fp8_status_t fp8_dequantize(const uint8_t* q, int64_t rows, int64_t cols, int64_t ldq,
+                            const float* s, int64_t s_stride_r, int64_t s_stride_c, int tile_rows,
+                            void* out, fp8_out_t out_type, int64_t ldo, fp8_stream_t stream) {
+    const int oes = elem_size_out(out_type);
+    if (oes == 0) return FP8_ERR_DTYPE;
+    if (rows < 0 || cols < 0 || cols % 128 != 0 || (tile_rows != 1 && tile_rows != 128))
+        return FP8_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return FP8_OK;
+    if (!q || !s || !out) return FP8_ERR_NULL;
+    if (ldq < cols || ldo < cols || s_stride_r < 0 || s_stride_c < 0) return FP8_ERR_LAYOUT;
+    if (!aligned16(q) || ldq % 16 != 0 || !aligned4(s) || !aligned16(out) || (ldo * oes) % 16 != 0)
+        return FP8_ERR_ALIGN;
+    int dev, sms;
+    fp8_status_t st = current_device(&dev, &sms);
+    if (st != FP8_OK) return st;
+    const int64_t gx = (cols + kDqCodesPerBlock - 1) / kDqCodesPerBlock;
+    // kDqBlocksPerSm resident blocks per SM, one wave.
+    int64_t gy = (static_cast<int64_t>(sms) * kDqBlocksPerSm + gx - 1) / gx;
+    if (gy > rows) gy = rows;
+    if (gy > 65535) gy = 65535;
+    const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
+    if (out_type == FP8_OUT_BF16)
+        dequant_kernel<true><<<grid, kDqThreads, 0, stream>>>(q, rows, cols, ldq, s, s_stride_r,
+                                                              s_stride_c, tile_rows, out, ldo);
+    else
+        dequant_kernel<false><<<grid, kDqThreads, 0, stream>>>(q, rows, cols, ldq, s, s_stride_r,
+                                                               s_stride_c, tile_rows, out, ldo);
+    return launch_status();
+}
 
 const char* fp8_status_string(fp8_status_t s) {
     switch (s) {

@@ -184,6 +184,32 @@ FP8FG_API fp8_status_t fp8_grouped_gemm(const uint8_t* a, int64_t lda, const flo
                               fp8_out_t c_type, int64_t ldc, const int32_t* offsets, int G,
                               int64_t total_M, int64_t N, int64_t K, fp8_stream_t stream);
 
+/*
+ * fp8_dequantize -- E4M3 codes back to real values.
+ * [HS] 2.2 (dequantize: code value times the tile's scale), the inverse
+ * direction of the two quantize calls above.
+ *
+ *     out[r, c] = E4M3(q[r, c]) * s[r / tile_rows, c / 128]
+ *
+ * one IEEE fp32 multiply, round to nearest; written as fp32, or as bf16
+ * (that fp32 value rounded to nearest even).  NaN codes give NaN.
+ *
+ *  q          device codes [rows, ldq]; 16-byte aligned, ldq % 16 == 0, ldq >= cols.
+ *  rows       >= 0, any value.  cols >= 0, a multiple of 128.
+ *  s          device fp32, s[(r / tile_rows) * s_stride_r + (c / 128) * s_stride_c]
+ *             (non-negative strides).
+ *  tile_rows  1 (activation tiles, sa [M, K/128]) or 128 (weight blocks,
+ *             sb [K/128, N/128]); anything else gives FP8_ERR_SHAPE.
+ *  out        device [rows, ldo] of out_type; 16-byte aligned,
+ *             ldo * sizeof(elem) % 16 == 0, ldo >= cols.
+ *  Errors: FP8_ERR_NULL, FP8_ERR_SHAPE, FP8_ERR_ALIGN, FP8_ERR_LAYOUT,
+ *          FP8_ERR_DTYPE, FP8_ERR_DEVICE, FP8_ERR_CUDA.
+ */
+FP8FG_API fp8_status_t fp8_dequantize(const uint8_t* q, int64_t rows, int64_t cols, int64_t ldq,
+                                      const float* s, int64_t s_stride_r, int64_t s_stride_c,
+                                      int tile_rows, void* out, fp8_out_t out_type, int64_t ldo,
+                                      fp8_stream_t stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 FP8FG_API const char* fp8_status_string(fp8_status_t status);
 

@@ -24,10 +24,10 @@ def L():
     return _lib.lib
 
 
-def test_header_declares_the_four_entry_points():
+def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("fp8_quantize_act_1x128", "fp8_quantize_weight_128x128", "fp8_blockscaled_gemm",
-              "fp8_grouped_gemm", "fp8_status_string", "fp8_get_device_error"):
+              "fp8_grouped_gemm", "fp8_dequantize", "fp8_status_string", "fp8_get_device_error"):
         assert n in names
 
 
@@ -149,3 +149,20 @@ def test_valid_arguments_without_gpu_report_device_error(L):
     assert gemm(L) == 6
     code = ctypes.c_int(0)
     assert L.fp8_get_device_error(None, ctypes.byref(code)) == 6
+
+
+def test_dequantize_argument_errors(L):
+    vp = ctypes.c_void_p
+    buf = ctypes.create_string_buffer(4096 + 16)
+    base = (ctypes.addressof(buf) + 15) // 16 * 16
+    p = vp(base)
+    # q, rows, cols, ldq, s, s_r, s_c, tile_rows, out, out_type, ldo, stream
+    assert L.fp8_dequantize(p, 4, 128, 128, p, 1, 1, 1, p, 5, 128, None) == 5      # dtype
+    assert L.fp8_dequantize(p, 4, 100, 128, p, 1, 1, 1, p, 0, 128, None) == 2      # cols % 128
+    assert L.fp8_dequantize(p, 4, 128, 128, p, 1, 1, 64, p, 0, 128, None) == 2     # tile_rows
+    assert L.fp8_dequantize(p, -1, 128, 128, p, 1, 1, 1, p, 0, 128, None) == 2     # rows < 0
+    assert L.fp8_dequantize(p, 0, 128, 128, None, 1, 1, 1, None, 0, 128, None) == 0  # empty: no-op
+    assert L.fp8_dequantize(None, 4, 128, 128, p, 1, 1, 1, p, 0, 128, None) == 1   # null
+    assert L.fp8_dequantize(p, 4, 128, 64, p, 1, 1, 1, p, 0, 128, None) == 4       # ldq < cols
+    assert L.fp8_dequantize(p, 4, 128, 136, p, 1, 1, 1, p, 0, 128, None) == 3      # ldq % 16
+    assert L.fp8_dequantize(vp(base + 8), 4, 128, 128, p, 1, 1, 1, p, 0, 128, None) == 3
