@@ -224,6 +224,77 @@ class FFN(Workload):
         return flops
 
 
+class FFNQuantOut(FFN):
+    """The FFN forward with its output quantized in the GEMM epilogue for the
+    next layer (E4M3 codes + 1x128 scales instead of a bf16 C)."""
+    name = "ffn_up_fwd_4096x18432x7168_fp8_out"
+    dominant = "blockscaled_gemm_quant"
+
+    def __init__(self, fp8, device, M=4096, K=7168, N=18432):
+        super().__init__(fp8, device, M, K, N)
+        self.kernels = ["quant_act_1x128", "quant_weight_128x128", "blockscaled_gemm_quant"]
+        if device is None:
+            return
+        del self.c
+        self.qc = torch.empty((M, N), dtype=torch.uint8, device=device)
+        self.sc = torch.empty((M, N // 128), dtype=torch.float32, device=device)
+
+    def config(self):
+        d = super().config()
+        d["workload"] = self.name
+        d["out"] = "E4M3 [%dx%d] + fp32 1x128 scales (quantized in the GEMM epilogue)" % (self.M, self.N)
+        return d
+
+    def algorithmic(self):
+        d = super().algorithmic()
+        d["blockscaled_gemm_quant"] = d.pop("blockscaled_gemm")
+        return d
+
+    def step(self, marks):
+        f = self.fp8
+        marks(0)
+        f.fp8_quantize_act_1x128(self.x, q=self.qx, sa=self.sx)
+        marks(1)
+        f.fp8_quantize_weight_128x128(self.w, transpose_out=True, q=self.qw, sb=self.sw)
+        marks(2)
+        f.fp8_blockscaled_gemm_quant(self.qx, self.sx, self.qw, self.sw, qc=self.qc, sc=self.sc)
+        marks(3)
+
+    def e2e_setup(self):
+        self.hx = self.x.cpu().pin_memory()
+        self.hw = self.w.cpu().pin_memory()
+        self.hqc = torch.empty((self.M, self.N), dtype=torch.uint8, pin_memory=True)
+        self.hsc = torch.empty((self.M, self.N // 128), dtype=torch.float32, pin_memory=True)
+        return self.hx.numel() * 2 + self.hw.numel() * 2, self.hqc.numel() + self.hsc.numel() * 4
+
+    def e2e_step(self):
+        f = self.fp8
+        x = self.hx.to("cuda", non_blocking=True)
+        w = self.hw.to("cuda", non_blocking=True)
+        qx, sx = f.fp8_quantize_act_1x128(x)
+        qw, sw = f.fp8_quantize_weight_128x128(w, transpose_out=True)
+        qc, sc = f.fp8_blockscaled_gemm_quant(qx, sx, qw, sw)
+        self.hqc.copy_(qc, non_blocking=True)
+        self.hsc.copy_(sc, non_blocking=True)
+
+    def oracle_sample(self, orc, rows, nbs):
+        """As FFN's, plus the 1x128 quantization of each sampled bf16 output block."""
+        xs = synth.ffn_inputs("cpu", M=self.M, K=self.K, N=self.N) if not hasattr(self, "_cpu") \
+            else self._cpu
+        self._cpu = xs
+        x, w = xs
+        xa = x[:rows].contiguous().view(torch.int16).numpy().view(np.uint16)
+        qa, sa = orc.quantize_act_1x128(xa)
+        flops = 0.0
+        for nb in range(nbs):
+            blk = w[:, nb * 128:(nb + 1) * 128].contiguous().view(torch.int16).numpy().view(np.uint16)
+            qb, sb = orc.quantize_weight_128x128(blk, transpose_out=True)
+            c_ref, _ = orc.gemm_ref(qa, sa, qb, sb, want_t=False)
+            orc.quantize_act_1x128(orc.f32_to_bf16_bits(c_ref.astype(np.float32)))
+            flops += 2.0 * rows * 128 * self.K
+        return flops
+
+
 class Quant(Workload):
     name = synth.QUANT.name
     unit = "GB/s"
@@ -540,12 +611,13 @@ class MoE(Workload):
         return flops
 
 
-WORKLOADS = {"ffn": FFN, "quant": Quant, "moe": MoE, "dgrad": DGrad, "dequant": Dequant}
+WORKLOADS = {"ffn": FFN, "ffn_q": FFNQuantOut, "quant": Quant, "moe": MoE, "dgrad": DGrad,
+             "dequant": Dequant}
 # Oracle sample per step: (rows, column blocks), sized for a few seconds per step.
-ORACLE_SAMPLE = {"ffn": (32, 2), "quant": (16, 4), "moe": (32, 1), "dgrad": (16, 1),
+ORACLE_SAMPLE = {"ffn": (32, 2), "ffn_q": (32, 2), "quant": (16, 4), "moe": (32, 1), "dgrad": (16, 1),
                  "dequant": (64, 8)}
 # The single CPU-baseline measurement of a run: about 10 s of oracle work.
-CPU_BASELINE_SAMPLE = {"ffn": (512, 36), "quant": (256, 72), "moe": (256, 12), "dgrad": (128, 8),
+CPU_BASELINE_SAMPLE = {"ffn": (512, 36), "ffn_q": (512, 36), "quant": (256, 72), "moe": (256, 12), "dgrad": (128, 8),
                        "dequant": (896, 120)}
 
 

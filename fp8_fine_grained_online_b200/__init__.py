@@ -128,6 +128,33 @@ def fp8_blockscaled_gemm(a, sa, b, sb, out_dtype=torch.bfloat16, c=None, sb_kb_n
     return c
 
 
+def fp8_blockscaled_gemm_quant(a, sa, b, sb, qc=None, sc=None, c=None, want_c=False,
+                               stream=None):
+    """Block-scaled GEMM with its output quantized for the next layer:
+    returns (qc uint8 [M, N] E4M3 codes, sc fp32 [M, N/128]) and, when
+    ``want_c`` (or ``c`` is given), the bf16 output [M, N] as a third value.
+    Bit-identical to fp8_blockscaled_gemm(..., bf16) + fp8_quantize_act_1x128."""
+    _rowmajor(a, "a")
+    _rowmajor(b, "b")
+    M, K = a.shape
+    N = b.shape[0]
+    if qc is None:
+        qc = torch.empty((M, N), dtype=torch.uint8, device=a.device)
+    if sc is None:
+        sc = torch.empty((M, N // 128), dtype=torch.float32, device=a.device)
+    if c is None and want_c:
+        c = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    if c is not None:
+        _rowmajor(c, "c")
+    st = _L.fp8_blockscaled_gemm_quant(
+        _ptr(a), a.stride(0), _ptr(sa), sa.stride(0), sa.stride(1), _ptr(b), b.stride(0), _ptr(sb),
+        sb.stride(0), sb.stride(1), _ptr(qc), qc.stride(0), _ptr(sc), sc.stride(0), sc.stride(1),
+        _ptr(c) if c is not None else None, c.stride(0) if c is not None else 0, M, N, K,
+        _stream(stream))
+    _lib.check(st, "fp8_blockscaled_gemm_quant")
+    return (qc, sc, c) if c is not None else (qc, sc)
+
+
 def fp8_grouped_gemm(a, sa, b, sb, offsets, out_dtype=torch.bfloat16, c=None, stream=None):
     """MoE grouped GEMM: a [total_M, K] rows sorted by group, b [G, N, K],
     sb [G, K/128, N/128], offsets int32 [G+1] on the device."""

@@ -70,9 +70,11 @@ fp8_status_t current_device(int* dev_out, int* sms_out) {
                     reinterpret_cast<const void*>(&blockscaled_gemm_pair_kernel<false, false>),
                     reinterpret_cast<const void*>(&blockscaled_gemm_pair_kernel<false, true>),
                     reinterpret_cast<const void*>(&blockscaled_gemm_pair_kernel<true, false>),
-                    reinterpret_cast<const void*>(&blockscaled_gemm_pair_kernel<true, true>)};
-                for (int i = 0; i < 4; ++i) {
-                    const size_t bytes = i < 2 ? kGemmPairSmemBytes : kGemmPairGroupedSmemBytes;
+                    reinterpret_cast<const void*>(&blockscaled_gemm_pair_kernel<true, true>),
+                    reinterpret_cast<const void*>(&blockscaled_gemm_pair_kernel<false, true, true>)};
+                for (int i = 0; i < 5; ++i) {
+                    const size_t bytes = (i == 2 || i == 3) ? kGemmPairGroupedSmemBytes
+                                                            : kGemmPairSmemBytes;
                     if (cudaFuncSetAttribute(pair_kernels[i],
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(bytes)) != cudaSuccess) {
@@ -265,7 +267,7 @@ fp8_status_t launch_quant_stream(const void* in, fp8_in_t t, int64_t ld, const Q
 }
 
 // Persistent CTA-pair GEMM: `pairs` clusters of 2 CTAs.
-template <bool kGrouped>
+template <bool kGrouped, bool kQuantOut = false>
 fp8_status_t launch_pair_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
                               int64_t pairs, fp8_out_t c_type, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
@@ -281,7 +283,9 @@ fp8_status_t launch_pair_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, co
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e;
-    if (c_type == FP8_OUT_BF16)
+    if (kQuantOut)
+        e = cudaLaunchKernelEx(&cfg, blockscaled_gemm_pair_kernel<kGrouped, true, true>, tmA, tmB, p);
+    else if (c_type == FP8_OUT_BF16)
         e = cudaLaunchKernelEx(&cfg, blockscaled_gemm_pair_kernel<kGrouped, true>, tmA, tmB, p);
     else
         e = cudaLaunchKernelEx(&cfg, blockscaled_gemm_pair_kernel<kGrouped, false>, tmA, tmB, p);
@@ -290,6 +294,43 @@ fp8_status_t launch_pair_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, co
         return FP8_ERR_CUDA;
     }
     return launch_status();
+}
+
+// Dense GEMM on CTA pairs after the argument checks; `out` carries the
+// output fields (c / ldc, or the quantized-output fields).
+template <bool kQuantOut>
+fp8_status_t dense_gemm(const uint8_t* a, int64_t lda, const float* sa, int64_t sa_stride_m,
+                        int64_t sa_stride_kb, const uint8_t* b, int64_t ldb, const float* sb,
+                        int64_t sb_stride_kb, int64_t sb_stride_nb, const GemmParams& out,
+                        fp8_out_t c_type, int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+    // 256 x 256 tiles, one per CTA pair (two SMs).
+    const int64_t num_mt = (M + kPairBM - 1) / kPairBM, num_nt = (N + kBN - 1) / kBN;
+    if (num_mt * num_nt > INT32_MAX || M > INT32_MAX) return FP8_ERR_SHAPE;
+    int dev, sms;
+    fp8_status_t st = current_device(&dev, &sms);
+    if (st != FP8_OK) return st;
+
+    CUtensorMap tmA, tmB;
+    const uint64_t kcols = static_cast<uint64_t>(K);
+    if (!make_operand_map(&tmA, a, static_cast<uint64_t>(M), kcols, static_cast<uint64_t>(lda), 128) ||
+        !make_operand_map(&tmB, b, static_cast<uint64_t>(N), kcols, static_cast<uint64_t>(ldb), 128))
+        return FP8_ERR_CUDA;
+
+    GemmParams p = out;
+    p.sa = sa; p.sa_sm = sa_stride_m; p.sa_skb = sa_stride_kb;
+    p.sb = sb; p.sb_sg = 0; p.sb_skb = sb_stride_kb; p.sb_snb = sb_stride_nb;
+    p.M = M; p.N = N;
+    p.nkb = static_cast<int>(K / 128);
+    p.num_mt = static_cast<int>(num_mt);
+    p.num_nt = static_cast<int>(num_nt);
+    // Bands of m-tiles whose A rows (band_m x 256 rows x K bytes) stay in
+    // L2 (about 40 MB of the 126 MB) while the pairs walk across N: B is
+    // then read from HBM once per band, A once.
+    const int64_t band = (int64_t{40} << 20) / (static_cast<int64_t>(kPairBM) * K);
+    p.band_m = static_cast<int>(band < 1 ? 1 : (band > num_mt ? num_mt : band));
+    p.offsets = nullptr; p.G = 1;
+    const int64_t pairs = grid_for(num_mt * num_nt, g_dev[dev].max_pairs, 1);
+    return launch_pair_gemm<false, kQuantOut>(tmA, tmB, p, pairs, c_type, stream);
 }
 
 }  // namespace
@@ -425,34 +466,38 @@ fp8_status_t fp8_blockscaled_gemm(const uint8_t* a, int64_t lda, const float* sa
     fp8_status_t st = check_gemm_common(a, lda, sa, sa_stride_m, sa_stride_kb, b, ldb, sb,
                                         sb_stride_kb, sb_stride_nb, c, c_type, ldc, N, K);
     if (st != FP8_OK) return st;
-    // 256 x 256 tiles, one per CTA pair (two SMs).
-    const int64_t num_mt = (M + kPairBM - 1) / kPairBM, num_nt = (N + kBN - 1) / kBN;
-    if (num_mt * num_nt > INT32_MAX || M > INT32_MAX) return FP8_ERR_SHAPE;
-    int dev, sms;
-    st = current_device(&dev, &sms);
+    GemmParams out{};
+    out.c = c; out.ldc = ldc;
+    return dense_gemm<false>(a, lda, sa, sa_stride_m, sa_stride_kb, b, ldb, sb, sb_stride_kb,
+                             sb_stride_nb, out, c_type, M, N, K, stream);
+}
+
+fp8_status_t fp8_blockscaled_gemm_quant(const uint8_t* a, int64_t lda, const float* sa,
+                                        int64_t sa_stride_m, int64_t sa_stride_kb,
+                                        const uint8_t* b, int64_t ldb, const float* sb,
+                                        int64_t sb_stride_kb, int64_t sb_stride_nb, uint8_t* qc,
+                                        int64_t ldqc, float* sc, int64_t sc_stride_m,
+                                        int64_t sc_stride_nb, void* c, int64_t ldc, int64_t M,
+                                        int64_t N, int64_t K, fp8_stream_t stream) {
+    if (M < 0 || N < 0 || K < 0 || N % 128 != 0 || K % 128 != 0) return FP8_ERR_SHAPE;
+    if (M == 0 || N == 0) return FP8_OK;
+    if (K == 0) return FP8_ERR_SHAPE;
+    if (!qc || !sc) return FP8_ERR_NULL;
+    if (ldqc < N || sc_stride_m < 0 || sc_stride_nb < 0 || (c && ldc < N)) return FP8_ERR_LAYOUT;
+    if (!aligned16(qc) || ldqc % 16 != 0 || !aligned4(sc) ||
+        (c && (!aligned16(c) || (ldc * 2) % 16 != 0)))
+        return FP8_ERR_ALIGN;
+    // The operand checks of the plain GEMM (a stand-in for c when c is null).
+    fp8_status_t st = check_gemm_common(a, lda, sa, sa_stride_m, sa_stride_kb, b, ldb, sb,
+                                        sb_stride_kb, sb_stride_nb, c ? c : static_cast<void*>(qc),
+                                        FP8_OUT_BF16, c ? ldc : N, N, K);
     if (st != FP8_OK) return st;
-
-    CUtensorMap tmA, tmB;
-    const uint64_t kcols = static_cast<uint64_t>(K);
-    if (!make_operand_map(&tmA, a, static_cast<uint64_t>(M), kcols, static_cast<uint64_t>(lda), 128) ||
-        !make_operand_map(&tmB, b, static_cast<uint64_t>(N), kcols, static_cast<uint64_t>(ldb), 128))
-        return FP8_ERR_CUDA;
-
-    GemmParams p{};
-    p.sa = sa; p.sa_sm = sa_stride_m; p.sa_skb = sa_stride_kb;
-    p.sb = sb; p.sb_sg = 0; p.sb_skb = sb_stride_kb; p.sb_snb = sb_stride_nb;
-    p.c = c; p.ldc = ldc; p.M = M; p.N = N;
-    p.nkb = static_cast<int>(K / 128);
-    p.num_mt = static_cast<int>(num_mt);
-    p.num_nt = static_cast<int>(num_nt);
-    // Bands of m-tiles whose A rows (band_m x 256 rows x K bytes) stay in
-    // L2 (about 40 MB of the 126 MB) while the pairs walk across N: B is
-    // then read from HBM once per band, A once.
-    const int64_t band = (int64_t{40} << 20) / (static_cast<int64_t>(kPairBM) * K);
-    p.band_m = static_cast<int>(band < 1 ? 1 : (band > num_mt ? num_mt : band));
-    p.offsets = nullptr; p.G = 1;
-    const int64_t pairs = grid_for(num_mt * num_nt, g_dev[dev].max_pairs, 1);
-    return launch_pair_gemm<false>(tmA, tmB, p, pairs, c_type, stream);
+    GemmParams out{};
+    out.c = c; out.ldc = ldc;
+    out.qc = qc; out.ldqc = ldqc;
+    out.sc = sc; out.sc_sm = sc_stride_m; out.sc_snb = sc_stride_nb;
+    return dense_gemm<true>(a, lda, sa, sa_stride_m, sa_stride_kb, b, ldb, sb, sb_stride_kb,
+                            sb_stride_nb, out, FP8_OUT_BF16, M, N, K, stream);
 }
 
 fp8_status_t fp8_grouped_gemm(const uint8_t* a, int64_t lda, const float* sa,

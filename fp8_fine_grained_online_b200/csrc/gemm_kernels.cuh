@@ -37,6 +37,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "quant_kernels.cuh"  // fused 1x128 quantization of the output
 #include "sm100_ptx.cuh"
 
 namespace fp8fg {
@@ -92,6 +93,12 @@ struct GemmParams {
     int band_m;      // dense raster: m-tiles per band
     const int32_t* offsets;  // grouped only: [G + 1]
     int G;
+    // Quantized output (fp8_blockscaled_gemm_quant): codes [M, ldqc] and
+    // scales sc[m * sc_sm + (n / 128) * sc_snb]; c (bf16) may then be null.
+    uint8_t* qc;
+    int64_t ldqc;
+    float* sc;
+    int64_t sc_sm, sc_snb;
 };
 
 // Grouped GEMM: the persistent tile schedule, built in shared memory from
@@ -260,7 +267,60 @@ __device__ __forceinline__ void promote32(float (&acc)[128], const uint32_t (&pa
 // the row slice.  `release(buf)` (called by lane 0 after the warp has read
 // its slice of a chunk) hands TMEM buffer `buf` back to the MMA issuer.
 // Returns false if a wait was abandoned because the CTA is aborting.
-template <bool kOutBf16, typename Release>
+// The row's 128 accumulators as the next layer's input: rounded to bf16
+// (stored as C when p.c is set), then quantized as one 1x128 activation tile
+// exactly as fp8_quantize_act_1x128 quantizes that bf16 row: NaN-skipping
+// amax, scale = amax / 448 (1 if 0), codes of the corrected quotient (exact
+// for bf16), IEEE division when the scale is off that path.
+__device__ __forceinline__ void store_row_quantized(const GemmParams& p, const float (&acc)[128],
+                                                    int64_t row, int64_t col0) {
+    uint32_t hb[64];
+#pragma unroll
+    for (int j = 0; j < 64; ++j) {
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * j], acc[2 * j + 1]);
+        hb[j] = *reinterpret_cast<const uint32_t*>(&b2);
+    }
+    uint32_t m = hb[0] & 0x7FFF7FFFu;
+#pragma unroll
+    for (int j = 1; j < 64; ++j) m = bf16x2_max(m, hb[j] & 0x7FFF7FFFu);
+    const float amax = fmaxf(__uint_as_float(m << 16), __uint_as_float(m & 0xFFFF0000u));
+    if (p.c != nullptr) {
+        uint4* out = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.c) + row * p.ldc + col0);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            out[j] = make_uint4(hb[4 * j], hb[4 * j + 1], hb[4 * j + 2], hb[4 * j + 3]);
+    }
+    const float s = scale_from_amax(amax);
+    const float r = __frcp_rn(s);
+    const uint64_t s2 = f2_pack(s, s);
+    const uint64_t neg_r2 = f2_pack(-r, -r);
+    const bool fast = corrected_path_ok(s);
+    uint4* qrow = reinterpret_cast<uint4*>(p.qc + row * p.ldqc + col0);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        uint2 codes[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            Raw8<uint16_t> raw;
+            raw.a = make_uint4(hb[8 * j + 4 * h], hb[8 * j + 4 * h + 1], hb[8 * j + 4 * h + 2],
+                               hb[8 * j + 4 * h + 3]);
+            if (fast) {
+                uint64_t n[4];
+                raw.to_neg_pairs(n);
+                codes[h] = encode8_corrected(n, s2, neg_r2);
+            } else {
+                float v[8];
+                raw.to_float(v);
+                codes[h].x = encode2_exact(v[0], v[1], s) | (encode2_exact(v[2], v[3], s) << 16);
+                codes[h].y = encode2_exact(v[4], v[5], s) | (encode2_exact(v[6], v[7], s) << 16);
+            }
+        }
+        qrow[j] = make_uint4(codes[0].x, codes[0].y, codes[1].x, codes[1].y);
+    }
+    p.sc[row * p.sc_sm + (col0 / 128) * p.sc_snb] = s;
+}
+
+template <bool kOutBf16, bool kQuantOut = false, typename Release>
 __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, uint64_t* tfull,
                                               volatile int* abort_flag, uint32_t tmem_base,
                                               uint32_t t_lane, int h, int lane, int64_t row,
@@ -321,7 +381,9 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, uint64_t* tfu
         promote32<96>(acc, pb, scale);
     }
     if (row_ok && col_ok) {
-        if (kOutBf16) {
+        if (kQuantOut) {
+            store_row_quantized(p, acc, row, col0);
+        } else if (kOutBf16) {
             __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.c) + row * p.ldc + col0;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {

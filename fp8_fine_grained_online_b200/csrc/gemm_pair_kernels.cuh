@@ -58,7 +58,7 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
     }
 }
 
-template <bool kGrouped, bool kOutBf16>
+template <bool kGrouped, bool kOutBf16, bool kQuantOut = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     blockscaled_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                                  const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
@@ -223,7 +223,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const bool row_ok = row < tc.row_end;
             const int64_t col0 = tc.n0 + h * 128;
             const bool col_ok = col0 < p.N;
-            ok = epilogue_tile<kOutBf16>(
+            ok = epilogue_tile<kOutBf16, kQuantOut>(
                 p, tail->tfull, abort_flag, tmem_base, t_lane, h, lane, row, row_ok, col0, col_ok,
                 tc.g, chunk, [&](uint32_t buf) { mbar_arrive_cluster(tempty_leader[buf]); });
         }

@@ -158,6 +158,33 @@ FP8FG_API fp8_status_t fp8_blockscaled_gemm(const uint8_t* a, int64_t lda, const
                                   fp8_stream_t stream);
 
 /*
+ * fp8_blockscaled_gemm_quant -- fp8_blockscaled_gemm whose output leaves
+ * already quantized for the next layer: the GEMM epilogue rounds each row
+ * of C to bf16 and quantizes every 1x128 tile of that bf16 row as
+ * fp8_quantize_act_1x128 does ([KB] "Finkornig kvantisering",
+ * "Online-kvantisering"), so codes and scales are bit-identical to
+ * fp8_blockscaled_gemm (bf16 out) followed by fp8_quantize_act_1x128 on C,
+ * without the round trip of C through memory.
+ *
+ *  a, sa, b, sb  as in fp8_blockscaled_gemm (b K-major, [N, ldb]).
+ *  qc     device codes [M, ldqc]; 16-byte aligned, ldqc % 16 == 0, ldqc >= N.
+ *  sc     device fp32, sc[m * sc_stride_m + (n / 128) * sc_stride_nb]
+ *         (e.g. [M, N/128] row-major: sc_stride_m = N/128, sc_stride_nb = 1).
+ *  c      optional device bf16 [M, ldc] copy of the rounded output (NULL: not
+ *         written); 16-byte aligned, ldc * 2 % 16 == 0, ldc >= N.
+ *  M >= 0 any value; N and K multiples of 128, K > 0 (K == 0: FP8_ERR_SHAPE).
+ *  Errors: as fp8_blockscaled_gemm.
+ */
+FP8FG_API fp8_status_t fp8_blockscaled_gemm_quant(const uint8_t* a, int64_t lda, const float* sa,
+                                                  int64_t sa_stride_m, int64_t sa_stride_kb,
+                                                  const uint8_t* b, int64_t ldb, const float* sb,
+                                                  int64_t sb_stride_kb, int64_t sb_stride_nb,
+                                                  uint8_t* qc, int64_t ldqc, float* sc,
+                                                  int64_t sc_stride_m, int64_t sc_stride_nb,
+                                                  void* c, int64_t ldc, int64_t M, int64_t N,
+                                                  int64_t K, fp8_stream_t stream);
+
+/*
  * fp8_grouped_gemm -- the block-scaled GEMM over MoE expert groups.
  * Same arithmetic as fp8_blockscaled_gemm ([KB] "Mixed Precision
  * Framework", "Ökad ackumuleringsprecision"), applied per expert g to the

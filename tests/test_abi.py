@@ -166,3 +166,24 @@ def test_dequantize_argument_errors(L):
     assert L.fp8_dequantize(p, 4, 128, 64, p, 1, 1, 1, p, 0, 128, None) == 4       # ldq < cols
     assert L.fp8_dequantize(p, 4, 128, 136, p, 1, 1, 1, p, 0, 128, None) == 3      # ldq % 16
     assert L.fp8_dequantize(vp(base + 8), 4, 128, 128, p, 1, 1, 1, p, 0, 128, None) == 3
+
+
+def test_gemm_quant_argument_errors(L):
+    vp = ctypes.c_void_p
+    buf = ctypes.create_string_buffer(4096 + 16)
+    base = (ctypes.addressof(buf) + 15) // 16 * 16
+    p = vp(base)
+
+    def call(qc=p, ldqc=128, sc=p, c=None, ldc=0, M=4, N=128, K=128):
+        # a, lda, sa, sa_m, sa_kb, b, ldb, sb, sb_kb, sb_nb, qc, ldqc, sc, sc_m, sc_nb, c, ldc, M, N, K
+        return L.fp8_blockscaled_gemm_quant(p, 128, p, 1, 1, p, 128, p, 1, 1, qc, ldqc, sc, 1, 1,
+                                            c, ldc, M, N, K, None)
+    assert call(N=100) == 2                 # N % 128
+    assert call(K=0) == 2                   # empty contraction not supported here
+    assert call(M=0, qc=None, sc=None) == 0  # empty: no-op
+    assert call(qc=None) == 1
+    assert call(sc=None) == 1
+    assert call(ldqc=64) == 4               # ldqc < N
+    assert call(ldqc=136) == 3              # ldqc % 16
+    assert call(c=p, ldc=64) == 4           # ldc < N
+    assert call(c=vp(base + 2), ldc=128) == 3
