@@ -89,6 +89,26 @@ def fp8_quantize_act_1x128(x, q=None, sa=None, stream=None):
     return q, sa
 
 
+def fp8_quantize_act_1x128_gather(x, rows, q=None, sa=None, stream=None):
+    """x [T, K] (bf16/fp32, CUDA), rows int32 [R] (CUDA) -> quantization of
+    x[rows]: (q uint8 [R, K], sa fp32 [R, K/128]), without forming x[rows]."""
+    _rowmajor(x, "x")
+    T, K = x.shape
+    if rows.dtype != torch.int32 or not rows.is_contiguous():
+        raise ValueError("rows must be a contiguous int32 tensor")
+    R = rows.shape[0]
+    if q is None:
+        q = torch.empty((R, K), dtype=torch.uint8, device=x.device)
+    if sa is None:
+        sa = torch.empty((R, K // 128), dtype=torch.float32, device=x.device)
+    _rowmajor(q, "q")
+    st = _L.fp8_quantize_act_1x128_gather(_ptr(x), _in_type(x), T, K, x.stride(0), _ptr(rows), R,
+                                          _ptr(q), q.stride(0), _ptr(sa), sa.stride(0),
+                                          sa.stride(1), _stream(stream))
+    _lib.check(st, "fp8_quantize_act_1x128_gather")
+    return q, sa
+
+
 def fp8_quantize_weight_128x128(w, transpose_out=True, q=None, sb=None, stream=None):
     """w [K, N] -> (q uint8 [N, K] if transpose_out else [K, N], sb fp32 [K/128, N/128])."""
     _rowmajor(w, "w")

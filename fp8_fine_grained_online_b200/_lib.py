@@ -24,6 +24,8 @@ _i64, _int, _vp = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
 SIGNATURES = {
     "fp8_quantize_act_1x128": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _i64, _vp, _i64, _i64,
                                       _vp]),
+    "fp8_quantize_act_1x128_gather": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _i64, _vp, _i64,
+                                             _vp, _i64, _i64, _vp]),
     "fp8_quantize_weight_128x128": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _int, _i64, _vp,
                                            _i64, _i64, _vp]),
     "fp8_blockscaled_gemm": (_int, [_vp, _i64, _vp, _i64, _i64, _vp, _i64, _int, _vp, _i64, _i64,

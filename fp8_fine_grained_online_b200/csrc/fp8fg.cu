@@ -17,6 +17,7 @@
 #include "quant_kernels.cuh"
 #include "quant_stream_kernels.cuh"
 #include "dequant_kernels.cuh"
+#include "quant_gather_kernels.cuh"
 
 namespace fp8fg {
 namespace {
@@ -339,6 +340,38 @@ fp8_status_t dense_gemm(const uint8_t* a, int64_t lda, const float* sa, int64_t 
 using namespace fp8fg;
 
 extern "C" {
+
+fp8_status_t fp8_quantize_act_1x128_gather(const void* x, fp8_in_t x_type, int64_t src_rows,
+                                           int64_t K, int64_t ldx, const int32_t* rows,
+                                           int64_t R, uint8_t* q, int64_t ldq, float* sa,
+                                           int64_t sa_stride_m, int64_t sa_stride_kb,
+                                           fp8_stream_t stream) {
+    const int es = elem_size_in(x_type);
+    if (es == 0) return FP8_ERR_DTYPE;
+    if (src_rows < 0 || R < 0 || K < 0 || K % 128 != 0) return FP8_ERR_SHAPE;
+    if (R == 0 || K == 0) return FP8_OK;
+    if (!x || !rows || !q || !sa) return FP8_ERR_NULL;
+    if (ldx < K || ldq < K || sa_stride_m < 0 || sa_stride_kb < 0) return FP8_ERR_LAYOUT;
+    if (!aligned16(x) || (ldx * es) % 16 != 0 || !aligned16(q) || ldq % 16 != 0 ||
+        !aligned4(sa) || !aligned4(rows))
+        return FP8_ERR_ALIGN;
+    int dev, sms;
+    fp8_status_t st = current_device(&dev, &sms);
+    if (st != FP8_OK) return st;
+    // one half-warp per output row at a time
+    const int64_t grid = grid_for((R + 15) / 16, sms, kGqMinBlocks);
+    const unsigned g = static_cast<unsigned>(grid);
+    const int64_t nkb = K / 128;
+    if (x_type == FP8_IN_BF16)
+        quant_gather_kernel<uint16_t><<<g, kGqThreads, 0, stream>>>(
+            static_cast<const uint16_t*>(x), src_rows, ldx, rows, R, nkb, q, ldq, sa, sa_stride_m,
+            sa_stride_kb);
+    else
+        quant_gather_kernel<float><<<g, kGqThreads, 0, stream>>>(
+            static_cast<const float*>(x), src_rows, ldx, rows, R, nkb, q, ldq, sa, sa_stride_m,
+            sa_stride_kb);
+    return launch_status();
+}
 
 fp8_status_t fp8_dequantize(const uint8_t* q, int64_t rows, int64_t cols, int64_t ldq,
                             const float* s, int64_t s_stride_r, int64_t s_stride_c, int tile_rows,

@@ -97,6 +97,27 @@ FP8FG_API fp8_status_t fp8_quantize_act_1x128(const void* x, fp8_in_t x_type, in
                                     fp8_stream_t stream);
 
 /*
+ * fp8_quantize_act_1x128_gather -- fp8_quantize_act_1x128 of a row gather:
+ * output row r is the 1x128 quantization of input row rows[r] (the MoE
+ * dispatch that sorts routed tokens by expert), bit-identical to gathering
+ * x[rows] first and quantizing that, without writing the gathered copy.
+ * [KB] "Finkornig kvantisering", "Online-kvantisering"; [HS] 2.2.
+ *
+ *  x        device [src_rows, ldx] of x_type; alignment as fp8_quantize_act_1x128.
+ *  rows     device int32 [R]: source row of each output row, 0 <= rows[r] <
+ *           src_rows.  An index out of range leaves that output row
+ *           unwritten and records FP8_ERR_SHAPE in the device error word.
+ *  q, sa    output [R, ldq] codes and sa[r * sa_stride_m + kb * sa_stride_kb],
+ *           as in fp8_quantize_act_1x128.
+ *  K        a multiple of 128.
+ */
+FP8FG_API fp8_status_t fp8_quantize_act_1x128_gather(const void* x, fp8_in_t x_type,
+                                                     int64_t src_rows, int64_t K, int64_t ldx,
+                                                     const int32_t* rows, int64_t R, uint8_t* q,
+                                                     int64_t ldq, float* sa, int64_t sa_stride_m,
+                                                     int64_t sa_stride_kb, fp8_stream_t stream);
+
+/*
  * fp8_quantize_weight_128x128 -- online fine-grained weight quantization.
  * [KB] "Finkornig kvantisering" (weights in 128x128 blocks, each scaled on
  * its own), "Online-kvantisering"; [HS] 2.2.

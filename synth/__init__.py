@@ -165,8 +165,9 @@ def moe_inputs(device="cpu", tokens=8192, experts=256, topk=8, hidden=7168, inte
                with_weights=True):
     """Routed activations and expert weights for the MoE grouped GEMMs.
 
-    Returns dict with: x_routed bf16 [tokens*topk, hidden] (rows sorted by
-    expert), offsets int32 [experts+1], h_down bf16 [tokens*topk, inter]
+    Returns dict with: x bf16 [tokens, hidden] (the tokens), x_routed bf16
+    [tokens*topk, hidden] (x[token_of]: rows sorted by expert), token_of int64
+    [tokens*topk], offsets int32 [experts+1], h_down bf16 [tokens*topk, inter]
     (input of the down projection, N(0,1)), and when ``with_weights``:
     w_gate_up bf16 [experts, hidden, 2*inter], w_down bf16 [experts, inter, hidden]
     (built expert by expert with ``moe_expert_weight``).
@@ -174,7 +175,7 @@ def moe_inputs(device="cpu", tokens=8192, experts=256, topk=8, hidden=7168, inte
     c = MOE.config_id
     x = act_input(tokens, hidden, 1.0, 1e-3, 100.0, c, device)
     token_of, offsets = moe_routing(tokens, experts, topk, seed_for(c, 2), device)
-    out = dict(x_routed=x[token_of].contiguous(), offsets=offsets, token_of=token_of)
+    out = dict(x=x, x_routed=x[token_of].contiguous(), offsets=offsets, token_of=token_of)
     out["h_down"] = normal((tokens * topk, inter), 1.0, seed_for(c, 3), device)
     if with_weights:
         out["w_gate_up"] = torch.stack([moe_expert_weight(e, "gate_up", device, hidden, inter)

@@ -187,3 +187,22 @@ def test_gemm_quant_argument_errors(L):
     assert call(ldqc=136) == 3              # ldqc % 16
     assert call(c=p, ldc=64) == 4           # ldc < N
     assert call(c=vp(base + 2), ldc=128) == 3
+
+
+def test_gather_quant_argument_errors(L):
+    vp = ctypes.c_void_p
+    buf = ctypes.create_string_buffer(4096 + 16)
+    base = (ctypes.addressof(buf) + 15) // 16 * 16
+    p = vp(base)
+
+    # x, x_type, src_rows, K, ldx, rows, R, q, ldq, sa, sa_m, sa_kb, stream
+    def call(x=p, xt=0, T=4, K=128, ldx=128, rows=p, R=4, q=p, ldq=128, sa=p):
+        return L.fp8_quantize_act_1x128_gather(x, xt, T, K, ldx, rows, R, q, ldq, sa, 1, 1, None)
+    assert call(xt=7) == 5
+    assert call(K=100) == 2
+    assert call(R=-1) == 2
+    assert call(R=0, x=None, rows=None, q=None, sa=None) == 0
+    assert call(rows=None) == 1
+    assert call(ldq=64) == 4
+    assert call(ldx=132) == 3          # ldx * 2 bytes % 16
+    assert call(rows=vp(base + 2)) == 3

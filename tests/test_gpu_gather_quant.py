@@ -1,0 +1,64 @@
+"""Fused row gather + 1x128 quantization (MoE dispatch): bit-identical to the
+oracle's quantization of the gathered rows x[rows]."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from _util import assert_codes_equal, assert_scales_equal, np_u8, to_oracle
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("T,R,K", [(1, 1, 128), (50, 77, 384), (300, 1201, 1024), (256, 2048, 7168)])
+def test_gather_quant_matches_oracle(cuda_lib, orc, T, R, K, dtype):
+    x = synth.act_input(T, K, 1.0, 1e-2, 100.0, 7, "cpu", dtype, tensor_id=T % 7)
+    g = torch.Generator().manual_seed(R)
+    rows = torch.randint(0, T, (R,), generator=g, dtype=torch.int32)
+    q, sa = cuda_lib.fp8_quantize_act_1x128_gather(x.cuda(), rows.cuda())
+    qo, sao = orc.quantize_act_1x128(to_oracle(x[rows.long()]))
+    assert_codes_equal(np_u8(q), qo)
+    assert_scales_equal(sa.cpu().numpy(), sao)
+
+
+def test_gather_quant_equals_gather_then_quantize(cuda_lib):
+    d = synth.moe_inputs("cpu", tokens=1024, experts=32, with_weights=False)
+    x = synth.act_input(1024, 7168, 1.0, 1e-3, 100.0, synth.MOE.config_id, "cpu").cuda()
+    rows = d["token_of"].to(torch.int32).cuda()
+    q1, s1 = cuda_lib.fp8_quantize_act_1x128_gather(x, rows)
+    q2, s2 = cuda_lib.fp8_quantize_act_1x128(x[rows.long()].contiguous())
+    assert torch.equal(q1, q2)
+    assert torch.equal(s1.view(torch.int32), s2.view(torch.int32))
+
+
+def test_invalid_index_reported_and_row_untouched(cuda_lib):
+    x = torch.randn(10, 256).bfloat16().cuda()
+    rows = torch.tensor([0, 3, 10, 9, -1], dtype=torch.int32).cuda()
+    q = torch.full((5, 256), 0xAB, dtype=torch.uint8, device="cuda")
+    sa = torch.full((5, 2), -3.0, device="cuda")
+    assert cuda_lib.fp8_get_device_error() == 0
+    cuda_lib.fp8_quantize_act_1x128_gather(x, rows, q=q, sa=sa)
+    assert cuda_lib.fp8_get_device_error() == 2
+    assert torch.all(q[2] == 0xAB) and torch.all(q[4] == 0xAB)
+    assert torch.all(sa[2] == -3.0) and torch.all(sa[4] == -3.0)
+    q_ok, s_ok = cuda_lib.fp8_quantize_act_1x128(x[[0, 3, 9]].contiguous())
+    assert torch.equal(q[[0, 1, 3]], q_ok)
+    assert torch.equal(sa[[0, 1, 3]], s_ok)
+
+
+@pytest.mark.slow
+def test_moe_dispatch_full_size_sampled(cuda_lib, orc):
+    """8192 tokens x top-8 of 256 experts: all 65536 routed rows equal the
+    unfused gather + quantize; sampled rows against the oracle."""
+    d = synth.moe_inputs("cpu", with_weights=False)
+    x = synth.act_input(8192, 7168, 1.0, 1e-3, 100.0, synth.MOE.config_id, "cpu")
+    rows = d["token_of"].to(torch.int32)
+    xc, rc = x.cuda(), rows.cuda()
+    q, sa = cuda_lib.fp8_quantize_act_1x128_gather(xc, rc)
+    q2, s2 = cuda_lib.fp8_quantize_act_1x128(xc[rc.long()].contiguous())
+    assert torch.equal(q, q2) and torch.equal(sa, s2)
+    pick = np.array([0, 1, 4095, 30000, 65535])
+    qo, sao = orc.quantize_act_1x128(to_oracle(x[rows[pick].long()]))
+    assert_codes_equal(np_u8(q[torch.from_numpy(pick).cuda()]), qo)
+    assert_scales_equal(sa[torch.from_numpy(pick).cuda()].cpu().numpy(), sao)
