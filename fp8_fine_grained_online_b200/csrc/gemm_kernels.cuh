@@ -26,7 +26,7 @@
 // Double-buffered TMEM lets the MMA of chunk kb+1 run while the epilogue
 // promotes chunk kb.
 //
-// Every mbarrier wait is bounded (kWaitLimitNs); on timeout the kernel
+// Every mbarrier wait is bounded (kWaitLimitCycles); on timeout the kernel
 // records FP8_ERR_DEVICE_TIMEOUT in the device error word, all roles stop,
 // in-flight copies and MMAs are waited for (bounded), TMEM is released and
 // the kernel returns.
@@ -65,7 +65,6 @@ constexpr int kBBytes = kBN * kBK;  // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kTmemCols = 512;      // 2 partial buffers x 256 FP32 columns
 constexpr int kMaxGroups = 1024;
-constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
 
 // Status codes recorded in the device error word (values of fp8_status_t).
 constexpr unsigned kDevErrShape = 2;
@@ -133,7 +132,7 @@ struct TileCoord {
 };
 
 // Wait for phase `parity` of `bar` to complete; false if this CTA aborted or
-// the wait ran past kWaitLimitNs (which aborts the CTA).
+// the wait ran past kWaitLimitCycles (which aborts the CTA).
 // The limit is counted in SM clock cycles (clock64 is a cheap local
 // counter; the device-wide %globaltimer is slow to read and would delay the
 // reaction to a completed barrier).  2^31 cycles is about one second at the

@@ -1,24 +1,26 @@
-// quant_stream_kernels.cuh -- online 128x128 weight quantization streamed
-// through shared memory by TMA.
-//
-// Every 128x128 block of w [K, N] gets scale = amax / 448 and codes
-// E4M3_RNE_satfinite(w / scale), bit-exact to IEEE fp32 division (see
-// encode8_bracket) (codingmall.com "Kan du förklara rollen för FP8 precision
-// i träningsprocessen för DeepSeek-V3", "Finkornig kvantisering",
+// quant_stream_kernels.cuh -- online fine-grained E4M3 quantization streamed
+// through shared memory by TMA, in three modes:
+//   activations: every 1x128 tile of x [M, K] gets its own scale;
+//   weights:     every 128x128 block of w [K, N] gets its own scale, codes
+//                written [K, N] as given, or transposed to [N, K] (K
+//                contiguous, the GEMM's B operand layout).
+// scale = amax / 448 and codes E4M3_RNE_satfinite(x / scale), bit-exact to
+// IEEE fp32 division (see encode8_corrected, encode8_bracket)
+// (codingmall.com "Kan du förklara rollen för FP8 precision i
+// träningsprocessen för DeepSeek-V3", "Finkornig kvantisering",
 // "Online-kvantisering"; holysheep.ai "FP8 混精度训练 DeepSeek 671B" (zh),
-// 2.2).  Output [K, N] as given, or transposed to [N, K] (K contiguous, the
-// GEMM's B operand layout).
+// 2.2).
 //
 // HBM-bound.  One persistent CTA per SM with two groups of 8 warps.  Group
 // g takes the CTA's boxes g, g+2, ... of 128x128 input elements; each group
 // owns two shared-memory slots (one for fp32 input) that its first thread
-// fills by TMA.  A block is read from shared memory twice (amax pass, then
-// encode pass); the slot is refilled with the group's box two ahead as soon
-// as the group has taken its second half into registers, so HBM reads
-// overlap the arithmetic of both groups.
+// fills by TMA; the slot is refilled with the group's box two ahead as soon
+// as the group has taken the box into registers (weights: its second half,
+// after the amax pass), so HBM reads overlap the arithmetic of both groups.
 //
 // Consumer thread (kq = t / 16, c = t % 16) of its group holds rows
-// {4kq .. 4kq+3, 64+4kq .. 64+4kq+3} of the box, columns [8c, 8c+8).
+// {4kq .. 4kq+3, 64+4kq .. 64+4kq+3} of the box, columns [8c, 8c+8): for
+// activations a half-warp holds 8 whole rows (8 tiles).
 #pragma once
 
 #include <cstdint>
