@@ -625,8 +625,8 @@ WORKLOADS = {"ffn": FFN, "ffn_q": FFNQuantOut, "quant": Quant, "moe": MoE, "dgra
 ORACLE_SAMPLE = {"ffn": (32, 2), "ffn_q": (32, 2), "quant": (16, 4), "moe": (32, 1), "dgrad": (16, 1),
                  "dequant": (64, 8)}
 # The single CPU-baseline measurement of a run: about 10 s of oracle work.
-CPU_BASELINE_SAMPLE = {"ffn": (512, 36), "ffn_q": (512, 36), "quant": (256, 72), "moe": (256, 12), "dgrad": (128, 8),
-                       "dequant": (896, 120)}
+CPU_BASELINE_SAMPLE = {"ffn": (1024, 60), "ffn_q": (1024, 60), "quant": (512, 144),
+                       "moe": (512, 24), "dgrad": (256, 24), "dequant": (896, 144)}
 
 
 # ----------------------------------------------------------------------------- timing
