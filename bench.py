@@ -85,14 +85,42 @@ def recorded_traffic(kernel, workload):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """SM clock and throttle reasons sampled during the timed region.
+
+    NVML (read-only queries) from a background thread every ~2 ms, so that
+    even a timed region of a few milliseconds gets several samples; the GPU
+    is found by its PCI address (robust to CUDA_VISIBLE_DEVICES).  Falls back
+    to `nvidia-smi -lms 100` when NVML is not importable."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    INTERVAL_S = 0.002
 
     def __init__(self, device_index):
+        import threading
         self.proc = None
-        self.idx = device_index
+        self.thread = None
+        self.samples = []
+        self.reasons = set()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            prop = torch.cuda.get_device_properties(device_index)
+            bus = "%08x:%02x:%02x.0" % (prop.pci_domain_id, prop.pci_bus_id, prop.pci_device_id)
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            self.reason_bits = {
+                "hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+            self.stop_flag = threading.Event()
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.thread = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
@@ -101,7 +129,33 @@ class ClockSampler:
         except (OSError, ValueError):
             self.proc = None
 
+    def _poll(self):
+        n = self.nvml
+        while not self.stop_flag.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM))
+                bits = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                for name, bit in self.reason_bits.items():
+                    if bits & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.INTERVAL_S)
+
+    def begin(self):
+        """Start of the timed region: drop samples taken before it."""
+        self.samples = []
+        self.reasons = set()
+
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=5)
+            if not self.samples:
+                return None
+            return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": float(self.max_mhz),
+                    "reasons": sorted(self.reasons), "samples": len(self.samples),
+                    "source": "nvml, every %.0f ms" % (self.INTERVAL_S * 1e3)}
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -127,7 +181,7 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi, every 100 ms"}
 
 
 # ----------------------------------------------------------------------------- workloads
@@ -681,6 +735,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     clocks = ClockSampler(torch.cuda.current_device())
     time.sleep(0.3)
+    clocks.begin()
     wall0 = time.perf_counter()
     start.record(stream)
     for s in range(args.steps):
@@ -688,8 +743,8 @@ def run_ours(args, rank, world, local_rank):
     stop.record(stream)
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
-    barrier()
     clk = clocks.stop()
+    barrier()
     elapsed_ms = max_over_ranks(start.elapsed_time(stop), world, device)
     dev_err = fp8.fp8_get_device_error()
 
