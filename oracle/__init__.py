@@ -228,3 +228,17 @@ def f32_to_bf16_bits(x):
     nan = np.isnan(np.asarray(x, dtype=np.float32))
     r[nan] = ((u[nan] >> 16) | 0x40).astype(np.uint16)
     return r
+
+
+def gemm_ref_colscale(qa, sa, qb, sb_cols):
+    """Block-scaled GEMM whose B scales are per output column and chunk (the
+    weight-gradient product dW = X^T dY, both operands quantized in 1x128
+    tiles along the contraction): C[i, n] = sum_k (sa[i, k/128] dec(qa[i, k]))
+    (sb_cols[n, k/128] dec(qb[n, k])), in fp64 (products of E4M3 values and
+    fp32 scales are exact there), and T = sum_k |.| of the same products
+    ([KB] "Ökad ackumuleringsprecision"; [HS] 2.2 dequantize).  qa [I, K],
+    qb [N, K] (K-major), sa [I, K/128], sb_cols [N, K/128].
+    Returns (C, T) as fp64 [I, N]."""
+    A = dequantize(qa, sa, 1, 128)
+    B = dequantize(qb, sb_cols, 1, 128)
+    return A @ B.T, np.abs(A) @ np.abs(B).T

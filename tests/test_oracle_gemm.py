@@ -128,3 +128,39 @@ def test_quantized_gemm_close_to_exact(orc):
     E = orc.gemm_exact(x, w)
     rel = np.linalg.norm(C - E) / np.linalg.norm(E)
     assert rel < 0.05
+
+
+def test_colscale_reduces_to_block_scales(orc):
+    """Per-column B scales that are equal within each 128-column block give
+    the block-scaled reference (a pinned function)."""
+    rng = np.random.default_rng(21)
+    I, N, K = 64, 256, 384
+    qa = rng.integers(0, 0x7E, (I, K)).astype(np.uint8)
+    qb = rng.integers(0, 0x7E, (N, K)).astype(np.uint8)
+    sa = rng.uniform(0.5, 2, (I, K // 128)).astype(np.float32)
+    sb_blk = rng.uniform(0.5, 2, (K // 128, N // 128)).astype(np.float32)
+    sb_cols = np.repeat(sb_blk.T, 128, axis=0)              # [N, K/128]
+    C1, T1 = orc.gemm_ref_colscale(qa, sa, qb, sb_cols)
+    C2, T2 = orc.gemm_ref(qa, sa, qb, sb_blk)
+    np.testing.assert_allclose(C1, C2, rtol=0, atol=1e-9 * np.max(T2))
+    np.testing.assert_allclose(T1, T2, rtol=1e-12)
+
+
+def test_colscale_closed_form_integers(orc):
+    """E4M3 small integers with power-of-two scales: every product and sum is
+    an exact integer multiple of a power of two, so C is known exactly."""
+    I, N, K = 8, 256, 256
+    codes = {1.0: 0x38, 2.0: 0x40, 3.0: 0x44, -1.0: 0xB8}
+    rng = np.random.default_rng(22)
+    va = rng.choice(list(codes), (I, K))
+    vb = rng.choice(list(codes), (N, K))
+    qa = np.vectorize(codes.get)(va).astype(np.uint8)
+    qb = np.vectorize(codes.get)(vb).astype(np.uint8)
+    sa = np.exp2(rng.integers(-3, 3, (I, K // 128))).astype(np.float32)
+    sb = np.exp2(rng.integers(-3, 3, (N, K // 128))).astype(np.float32)
+    C, _ = orc.gemm_ref_colscale(qa, sa, qb, sb)
+    ref = np.zeros((I, N))
+    for kb in range(K // 128):
+        blk = slice(kb * 128, (kb + 1) * 128)
+        ref += (va[:, blk] * sa[:, kb:kb + 1]) @ (vb[:, blk] * sb[:, kb:kb + 1]).T
+    assert np.array_equal(C, ref)
