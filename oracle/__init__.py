@@ -99,6 +99,15 @@ def quantize_act_1x128(x):
     return q, sa
 
 
+def quantize_act_128x1(x):
+    """x [M,K] -> (qt uint8 [K,M], st float32 [K, ceil(M/128)]): the 1x128
+    activation quantization ([KB] "Finkornig kvantisering") of x^T, i.e.
+    tiles of 128 consecutive rows of one column of x, as the weight gradient
+    X^T dY needs for its contraction over the rows (tokens)."""
+    x, _ = _as_input(x)
+    return quantize_act_1x128(np.ascontiguousarray(x.T))
+
+
 def quantize_weight_128x128(w, transpose_out=False):
     """w [K,N] -> (q uint8 [K,N] or [N,K], sb float32 [ceil(K/128), ceil(N/128)])."""
     w, t = _as_input(w)

@@ -179,6 +179,37 @@ def test_act_bf16_matches_fp32_of_same_values(orc):
 # weight quantizer
 # ----------------------------------------------------------------------------
 
+# ----------------------------------------------------------------------------
+# 128x1 activation quantizer (1x128 tiles of X^T, for the weight gradient)
+# ----------------------------------------------------------------------------
+
+def test_act_128x1_scale_is_column_amax_over_448(orc):
+    """st[k, mb] = fl32(max over rows 128 mb .. 128 mb + 127 of |x[m, k]| / 448),
+    computed here along the columns of x directly."""
+    x = as_np(rand_act(384, 256, 61))
+    qt, st = orc.quantize_act_128x1(x)
+    assert qt.shape == (256, 384) and st.shape == (256, 3)
+    amax = np.max(np.abs(values(x).reshape(3, 128, 256)), axis=1).astype(np.float32)   # [mb, k]
+    assert np.array_equal(st, (amax / np.float32(448.0)).T)
+
+
+def test_act_128x1_codes_exact_quotient_then_torch_cast(orc):
+    """qt[k, m] = cast(RN_fp32(x[m, k] / st[k, m / 128])), with the quotient
+    from fp64 division and PyTorch's E4M3 cast; a column's largest element
+    maps to +-448."""
+    x = as_np(rand_act(256, 384, 71))
+    qt, st = orc.quantize_act_128x1(x)
+    v = values(x).astype(np.float64)                       # [m, k]
+    s = np.repeat(st.T, 128, axis=0).astype(np.float64)    # [m, k]
+    quot = (v / s).astype(np.float32)
+    ref = torch.from_numpy(quot).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(qt, ref.T)
+    blocks = np.abs(values(x)).reshape(2, 128, 384)
+    top = blocks == blocks.max(axis=1, keepdims=True)
+    codes = qt.T.reshape(2, 128, 384)
+    assert np.all((codes[top] & 0x7F) == 0x7E)
+
+
 def rand_weight(K, N, seed, dtype=torch.bfloat16):
     w = normal((K, N), 0.02, seed, "cpu", dtype)
     set_outliers(w, 1e-3, 1.0, seed + 1, seed + 2)
