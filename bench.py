@@ -14,6 +14,11 @@ Workloads (``--workload``):
          weights are quantized once before timing.  value in TFLOP/s.
   dgrad  backward dgrad: dY bf16 [16384x18432] quantized 1x128 along N, W
          [7168x18432] quantized (untransposed), dX = dY W^T -> bf16.
+  wgrad  backward wgrad: X bf16 [16384x7168] and dY bf16 [16384x18432]
+         quantized in 1x128 tiles along the 16384 tokens (written transposed),
+         dW = X^T dY -> fp32 [7168x18432] by the GEMM with per-column B scales.
+  ffn_q  ffn with the GEMM's output quantized 1x128 in its epilogue.
+  dequant  the FFN weight's codes back to bf16.
 
 Contract: ``python bench.py --gpus N --steps K --warmup W`` (N > 1 under
 torchrun, one rank per GPU) prints one JSON line on rank 0.  Each rank runs
@@ -551,6 +556,88 @@ class DGrad(FFN):
         return flops
 
 
+class WGrad(Workload):
+    """dW = X^T dY: X and dY quantized in 1x128 tiles along the tokens (the
+    contraction), written transposed; the GEMM with per-column B scales."""
+    name = synth.WGRAD.name
+    unit = "TFLOP/s"
+    dominant = "blockscaled_gemm_colscale"
+    sample_text = ("%d rows x %d 128-column blocks of dW, with the 128x1 quantization of the "
+                   "X and dY columns they use")
+
+    def __init__(self, fp8, device, M=16384, K=7168, N=18432):
+        self.fp8, self.M, self.K, self.N = fp8, M, K, N
+        self.kernels = ["quant_act_128x1_x", "quant_act_128x1_dy", "blockscaled_gemm_colscale"]
+        if device is None:
+            return
+        self.x, self.dy = synth.wgrad_inputs(device, M, K, N)      # [M, K], [M, N]
+        self.qxt = torch.empty((K, M), dtype=torch.uint8, device=device)
+        self.sxt = torch.empty((K, M // 128), dtype=torch.float32, device=device)
+        self.qdt = torch.empty((N, M), dtype=torch.uint8, device=device)
+        self.sdt = torch.empty((M // 128, N), dtype=torch.float32, device=device)
+        self.c = torch.empty((K, N), dtype=torch.float32, device=device)
+
+    def config(self):
+        return {"workload": self.name, "tokens": self.M, "K": self.K, "N": self.N,
+                "x": "bf16 [%dx%d] N(0,1) 0.1%% outliers x100" % (self.M, self.K),
+                "dy": "bf16 [%dx%d] N(0,1e-3) 0.1%% outliers x100" % (self.M, self.N),
+                "out": "fp32 dW [%dx%d]" % (self.K, self.N),
+                "l2": "inputs larger than L2 (X+dY bf16 = %.0f MB > 126 MB)" %
+                      ((self.M * self.K + self.M * self.N) * 2 / 1e6)}
+
+    def flops(self):
+        return 2.0 * self.M * self.N * self.K
+
+    def work_per_step(self):
+        return self.flops()
+
+    def algorithmic(self):
+        M, N, K = self.M, self.N, self.K
+        return {
+            "quant_act_128x1_x": ("bytes", M * K * 2 + M * K + (M // 128) * K * 4),
+            "quant_act_128x1_dy": ("bytes", M * N * 2 + M * N + (M // 128) * N * 4),
+            "blockscaled_gemm_colscale": ("flops", 2.0 * M * N * K),
+        }
+
+    def step(self, marks):
+        f = self.fp8
+        marks(0)
+        f.fp8_quantize_act_128x1(self.x, qt=self.qxt, st=self.sxt)
+        marks(1)
+        f.fp8_quantize_act_128x1(self.dy, qt=self.qdt, st=self.sdt, st_kb_major=True)
+        marks(2)
+        f.fp8_blockscaled_gemm_colscale(self.qxt, self.sxt, self.qdt, self.sdt, c=self.c)
+        marks(3)
+
+    def e2e_setup(self):
+        self.hx = self.x.cpu().pin_memory()
+        self.hdy = self.dy.cpu().pin_memory()
+        self.hc = torch.empty((self.K, self.N), dtype=torch.float32, pin_memory=True)
+        return (self.hx.numel() + self.hdy.numel()) * 2, self.hc.numel() * 4
+
+    def e2e_step(self):
+        x = self.hx.to("cuda", non_blocking=True)
+        dy = self.hdy.to("cuda", non_blocking=True)
+        self.hc.copy_(self.fp8.linear_weight_grad(x, dy), non_blocking=True)
+
+    def oracle_sample(self, orc, rows, nbs):
+        """dW rows 0..rows-1 (columns of X) x the first nbs 128-column blocks
+        (columns of dY), each column quantized 128x1 over all tokens."""
+        if not hasattr(self, "_cpu"):
+            self._cpu = synth.wgrad_inputs("cpu", self.M, self.K, self.N)
+        x, dy = self._cpu
+        xa = x[:, :rows].contiguous().view(torch.int16).numpy().view(np.uint16)
+        qa, sa = orc.quantize_act_128x1(xa)
+        flops = 0.0
+        for nb in range(nbs):
+            blk = dy[:, nb * 128:(nb + 1) * 128].contiguous().view(torch.int16).numpy() \
+                .view(np.uint16)
+            qb, sb = orc.quantize_act_128x1(blk)
+            orc.gemm_ref_colscale(qa, sa, qb, sb)
+            flops += 2.0 * rows * 128 * self.M
+        return flops
+
+
 class MoE(Workload):
     name = synth.MOE.name
     unit = "TFLOP/s"
@@ -674,13 +761,14 @@ class MoE(Workload):
 
 
 WORKLOADS = {"ffn": FFN, "ffn_q": FFNQuantOut, "quant": Quant, "moe": MoE, "dgrad": DGrad,
-             "dequant": Dequant}
+             "dequant": Dequant, "wgrad": WGrad}
 # Oracle sample per step: (rows, column blocks), sized for a few seconds per step.
 ORACLE_SAMPLE = {"ffn": (32, 2), "ffn_q": (32, 2), "quant": (16, 4), "moe": (32, 1), "dgrad": (16, 1),
-                 "dequant": (64, 8)}
+                 "dequant": (64, 8), "wgrad": (16, 1)}
 # The single CPU-baseline measurement of a run: about 10 s of oracle work.
 CPU_BASELINE_SAMPLE = {"ffn": (1024, 60), "ffn_q": (1024, 60), "quant": (512, 144),
-                       "moe": (512, 24), "dgrad": (256, 24), "dequant": (896, 144)}
+                       "moe": (512, 24), "dgrad": (256, 24), "dequant": (896, 144),
+                       "wgrad": (512, 24)}
 
 
 # ----------------------------------------------------------------------------- timing

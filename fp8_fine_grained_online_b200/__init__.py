@@ -26,7 +26,9 @@ from ._lib import (FP8_IN_BF16, FP8_IN_FP32, FP8_OUT_BF16, FP8_OUT_FP32, LIB_PAT
 __all__ = [
     "fp8_quantize_act_1x128", "fp8_quantize_weight_128x128", "fp8_blockscaled_gemm",
     "fp8_grouped_gemm", "fp8_status_string", "fp8_get_device_error", "Fp8Error",
-    "LIB_PATH", "linear_forward", "e2e_linear_forward",
+    "LIB_PATH", "linear_forward", "e2e_linear_forward", "fp8_quantize_act_1x128_gather",
+    "fp8_blockscaled_gemm_quant", "fp8_dequantize", "fp8_quantize_act_128x1",
+    "fp8_blockscaled_gemm_colscale", "linear_weight_grad",
 ]
 
 _L = _lib.lib
@@ -173,6 +175,54 @@ def fp8_blockscaled_gemm_quant(a, sa, b, sb, qc=None, sc=None, c=None, want_c=Fa
         _stream(stream))
     _lib.check(st, "fp8_blockscaled_gemm_quant")
     return (qc, sc, c) if c is not None else (qc, sc)
+
+
+def fp8_quantize_act_128x1(x, qt=None, st=None, st_kb_major=False, stream=None):
+    """x [M, K] (bf16, CUDA) -> 1x128 quantization of x^T along M:
+    (qt uint8 [K, M] E4M3 codes, st fp32 scales), st [K, M/128] or, with
+    ``st_kb_major``, [M/128, K] (the layout of the column-scale GEMM's sb)."""
+    _rowmajor(x, "x")
+    M, K = x.shape
+    if qt is None:
+        qt = torch.empty((K, M), dtype=torch.uint8, device=x.device)
+    if st is None:
+        shape = (M // 128, K) if st_kb_major else (K, M // 128)
+        st = torch.empty(shape, dtype=torch.float32, device=x.device)
+    _rowmajor(qt, "qt")
+    s_k, s_mb = (st.stride(1), st.stride(0)) if st_kb_major else (st.stride(0), st.stride(1))
+    status = _L.fp8_quantize_act_128x1(_ptr(x), _in_type(x), M, K, x.stride(0), _ptr(qt),
+                                       qt.stride(0), _ptr(st), s_k, s_mb, _stream(stream))
+    _lib.check(status, "fp8_quantize_act_128x1")
+    return qt, st
+
+
+def fp8_blockscaled_gemm_colscale(a, sa, b, sb, out_dtype=torch.bfloat16, c=None, stream=None):
+    """C [M, N] = a [M, K] x b^T (b [N, K]) with 1x128 scales on both
+    operands: sa [M, K/128] indexed [m, kb], sb [K/128, N] indexed [kb, n]."""
+    _rowmajor(a, "a")
+    _rowmajor(b, "b")
+    _rowmajor(sb, "sb")
+    M, K = a.shape
+    N = b.shape[0]
+    if c is None:
+        c = torch.empty((M, N), dtype=out_dtype, device=a.device)
+    _rowmajor(c, "c")
+    st = _L.fp8_blockscaled_gemm_colscale(_ptr(a), a.stride(0), _ptr(sa), sa.stride(0),
+                                          sa.stride(1), _ptr(b), b.stride(0), _ptr(sb),
+                                          sb.stride(0), _ptr(c), _out_type(c.dtype), c.stride(0),
+                                          M, N, K, _stream(stream))
+    _lib.check(st, "fp8_blockscaled_gemm_colscale")
+    return c
+
+
+def linear_weight_grad(x, dy, out_dtype=torch.float32, stream=None):
+    """Weight gradient of y = x @ w in FP8: dW [K, N] = x^T dy with x [M, K],
+    dy [M, N] (bf16).  Both are quantized in 1x128 tiles along the tokens M
+    (scales computed on this call), then multiplied by the column-scale GEMM.
+    Three library calls."""
+    qxt, sxt = fp8_quantize_act_128x1(x, stream=stream)
+    qdt, sdt = fp8_quantize_act_128x1(dy, st_kb_major=True, stream=stream)
+    return fp8_blockscaled_gemm_colscale(qxt, sxt, qdt, sdt, out_dtype=out_dtype, stream=stream)
 
 
 def fp8_grouped_gemm(a, sa, b, sb, offsets, out_dtype=torch.bfloat16, c=None, stream=None):

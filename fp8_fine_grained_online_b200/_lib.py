@@ -33,6 +33,10 @@ SIGNATURES = {
     "fp8_blockscaled_gemm_quant": (_int, [_vp, _i64, _vp, _i64, _i64, _vp, _i64, _vp, _i64, _i64,
                                           _vp, _i64, _vp, _i64, _i64, _vp, _i64, _i64, _i64,
                                           _i64, _vp]),
+    "fp8_quantize_act_128x1": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _i64, _vp, _i64, _i64,
+                                      _vp]),
+    "fp8_blockscaled_gemm_colscale": (_int, [_vp, _i64, _vp, _i64, _i64, _vp, _i64, _vp, _i64,
+                                             _vp, _int, _i64, _i64, _i64, _i64, _vp]),
     "fp8_grouped_gemm": (_int, [_vp, _i64, _vp, _i64, _i64, _vp, _i64, _vp, _i64, _i64, _i64,
                                 _vp, _int, _i64, _vp, _int, _i64, _i64, _i64, _vp]),
     "fp8_dequantize": (_int, [_vp, _i64, _i64, _i64, _vp, _i64, _i64, _int, _vp, _int, _i64,

@@ -72,9 +72,12 @@ fp8_status_t current_device(int* dev_out, int* sms_out) {
                     reinterpret_cast<const void*>(&blockscaled_gemm_pair_kernel<false, true>),
                     reinterpret_cast<const void*>(&blockscaled_gemm_pair_kernel<true, false>),
                     reinterpret_cast<const void*>(&blockscaled_gemm_pair_kernel<true, true>),
-                    reinterpret_cast<const void*>(&blockscaled_gemm_pair_kernel<false, true, true>)};
-                for (int i = 0; i < 5; ++i) {
+                    reinterpret_cast<const void*>(&blockscaled_gemm_pair_kernel<false, true, true>),
+                    reinterpret_cast<const void*>(&blockscaled_gemm_pair_kernel<false, false, false, true>),
+                    reinterpret_cast<const void*>(&blockscaled_gemm_pair_kernel<false, true, false, true>)};
+                for (int i = 0; i < 7; ++i) {
                     const size_t bytes = (i == 2 || i == 3) ? kGemmPairGroupedSmemBytes
+                                         : i >= 5           ? kGemmPairColScaleSmemBytes
                                                             : kGemmPairSmemBytes;
                     if (cudaFuncSetAttribute(pair_kernels[i],
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -89,14 +92,16 @@ fp8_status_t current_device(int* dev_out, int* sms_out) {
                     reinterpret_cast<const void*>(&quant_stream_kernel<uint16_t, kQuantWeightT>),
                     reinterpret_cast<const void*>(&quant_stream_kernel<float, kQuantAct>),
                     reinterpret_cast<const void*>(&quant_stream_kernel<float, kQuantWeight>),
-                    reinterpret_cast<const void*>(&quant_stream_kernel<float, kQuantWeightT>)};
+                    reinterpret_cast<const void*>(&quant_stream_kernel<float, kQuantWeightT>),
+                    reinterpret_cast<const void*>(&quant_stream_kernel<uint16_t, kQuantActT>)};
                 const size_t qs_bytes[] = {quant_stream_smem_bytes<uint16_t, kQuantAct>(),
                                            quant_stream_smem_bytes<uint16_t, kQuantWeight>(),
                                            quant_stream_smem_bytes<uint16_t, kQuantWeightT>(),
                                            quant_stream_smem_bytes<float, kQuantAct>(),
                                            quant_stream_smem_bytes<float, kQuantWeight>(),
-                                           quant_stream_smem_bytes<float, kQuantWeightT>()};
-                for (int i = 0; i < 6; ++i) {
+                                           quant_stream_smem_bytes<float, kQuantWeightT>(),
+                                           quant_stream_smem_bytes<uint16_t, kQuantActT>()};
+                for (int i = 0; i < 7; ++i) {
                     if (cudaFuncSetAttribute(qs_kernels[i],
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(qs_bytes[i])) != cudaSuccess) {
@@ -258,6 +263,8 @@ fp8_status_t launch_quant_stream(const void* in, fp8_in_t t, int64_t ld, const Q
         return FP8_ERR_CUDA;
     if (t == FP8_IN_BF16) {
         if (mode == kQuantAct) return launch_quant_stream_t<uint16_t, kQuantAct>(map, p, sms, stream);
+        if (mode == kQuantActT)
+            return launch_quant_stream_t<uint16_t, kQuantActT>(map, p, sms, stream);
         if (mode == kQuantWeight)
             return launch_quant_stream_t<uint16_t, kQuantWeight>(map, p, sms, stream);
         return launch_quant_stream_t<uint16_t, kQuantWeightT>(map, p, sms, stream);
@@ -268,13 +275,15 @@ fp8_status_t launch_quant_stream(const void* in, fp8_in_t t, int64_t ld, const Q
 }
 
 // Persistent CTA-pair GEMM: `pairs` clusters of 2 CTAs.
-template <bool kGrouped, bool kQuantOut = false>
+template <bool kGrouped, bool kQuantOut = false, bool kColScaleB = false>
 fp8_status_t launch_pair_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
                               int64_t pairs, fp8_out_t c_type, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
     cfg.blockDim = dim3(kGemmThreads, 1, 1);
-    cfg.dynamicSmemBytes = kGrouped ? kGemmPairGroupedSmemBytes : kGemmPairSmemBytes;
+    cfg.dynamicSmemBytes = kGrouped     ? kGemmPairGroupedSmemBytes
+                           : kColScaleB ? kGemmPairColScaleSmemBytes
+                                        : kGemmPairSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -284,7 +293,11 @@ fp8_status_t launch_pair_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, co
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e;
-    if (kQuantOut)
+    if (kColScaleB && !kGrouped && c_type == FP8_OUT_BF16)
+        e = cudaLaunchKernelEx(&cfg, blockscaled_gemm_pair_kernel<false, true, false, true>, tmA, tmB, p);
+    else if (kColScaleB && !kGrouped)
+        e = cudaLaunchKernelEx(&cfg, blockscaled_gemm_pair_kernel<false, false, false, true>, tmA, tmB, p);
+    else if (kQuantOut)
         e = cudaLaunchKernelEx(&cfg, blockscaled_gemm_pair_kernel<kGrouped, true, true>, tmA, tmB, p);
     else if (c_type == FP8_OUT_BF16)
         e = cudaLaunchKernelEx(&cfg, blockscaled_gemm_pair_kernel<kGrouped, true>, tmA, tmB, p);
@@ -299,7 +312,7 @@ fp8_status_t launch_pair_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, co
 
 // Dense GEMM on CTA pairs after the argument checks; `out` carries the
 // output fields (c / ldc, or the quantized-output fields).
-template <bool kQuantOut>
+template <bool kQuantOut, bool kColScaleB = false>
 fp8_status_t dense_gemm(const uint8_t* a, int64_t lda, const float* sa, int64_t sa_stride_m,
                         int64_t sa_stride_kb, const uint8_t* b, int64_t ldb, const float* sb,
                         int64_t sb_stride_kb, int64_t sb_stride_nb, const GemmParams& out,
@@ -331,7 +344,7 @@ fp8_status_t dense_gemm(const uint8_t* a, int64_t lda, const float* sa, int64_t 
     p.band_m = static_cast<int>(band < 1 ? 1 : (band > num_mt ? num_mt : band));
     p.offsets = nullptr; p.G = 1;
     const int64_t pairs = grid_for(num_mt * num_nt, g_dev[dev].max_pairs, 1);
-    return launch_pair_gemm<false, kQuantOut>(tmA, tmB, p, pairs, c_type, stream);
+    return launch_pair_gemm<false, kQuantOut, kColScaleB>(tmA, tmB, p, pairs, c_type, stream);
 }
 
 }  // namespace
@@ -531,6 +544,55 @@ fp8_status_t fp8_blockscaled_gemm_quant(const uint8_t* a, int64_t lda, const flo
     out.sc = sc; out.sc_sm = sc_stride_m; out.sc_snb = sc_stride_nb;
     return dense_gemm<true>(a, lda, sa, sa_stride_m, sa_stride_kb, b, ldb, sb, sb_stride_kb,
                             sb_stride_nb, out, FP8_OUT_BF16, M, N, K, stream);
+}
+
+fp8_status_t fp8_quantize_act_128x1(const void* x, fp8_in_t x_type, int64_t M, int64_t K,
+                                    int64_t ldx, uint8_t* qt, int64_t ldq, float* st,
+                                    int64_t st_stride_k, int64_t st_stride_mb,
+                                    fp8_stream_t stream) {
+    const int es = elem_size_in(x_type);
+    if (es == 0) return FP8_ERR_DTYPE;
+    if (M < 0 || K < 0 || M % 128 != 0 || K % 128 != 0) return FP8_ERR_SHAPE;
+    if (M == 0 || K == 0) return FP8_OK;
+    if (x_type != FP8_IN_BF16) return FP8_ERR_DTYPE;
+    if (!x || !qt || !st) return FP8_ERR_NULL;
+    if (ldx < K || ldq < M || st_stride_k < 0 || st_stride_mb < 0) return FP8_ERR_LAYOUT;
+    if (!aligned16(x) || (ldx * es) % 16 != 0 || !aligned16(qt) || ldq % 16 != 0 || !aligned4(st))
+        return FP8_ERR_ALIGN;
+    if (M > INT32_MAX || K > INT32_MAX) return FP8_ERR_SHAPE;
+    int dev, sms;
+    fp8_status_t s = current_device(&dev, &sms);
+    if (s != FP8_OK) return s;
+    QsParams p{};
+    p.rows = M; p.cols = K;
+    p.nbr = M / 128; p.nbc = K / 128;
+    p.q = qt; p.ldq = ldq;
+    p.s = st; p.s_stride_r = st_stride_k; p.s_stride_c = st_stride_mb;
+    return launch_quant_stream(x, x_type, ldx, p, kQuantActT, sms, stream);
+}
+
+fp8_status_t fp8_blockscaled_gemm_colscale(const uint8_t* a, int64_t lda, const float* sa,
+                                           int64_t sa_stride_m, int64_t sa_stride_kb,
+                                           const uint8_t* b, int64_t ldb, const float* sb,
+                                           int64_t sb_stride_kb, void* c, fp8_out_t c_type,
+                                           int64_t ldc, int64_t M, int64_t N, int64_t K,
+                                           fp8_stream_t stream) {
+    if (elem_size_out(c_type) == 0) return FP8_ERR_DTYPE;
+    if (M < 0 || N < 0 || K < 0 || N % 128 != 0 || K % 128 != 0) return FP8_ERR_SHAPE;
+    if (M == 0 || N == 0) return FP8_OK;
+    if (K == 0) return zero_output(c, c_type, ldc, M, N, stream);
+    fp8_status_t st = check_gemm_common(a, lda, sa, sa_stride_m, sa_stride_kb, b, ldb, sb,
+                                        sb_stride_kb, 1, c, c_type, ldc, N, K);
+    if (st != FP8_OK) return st;
+    // Each epilogue warp copies its 128 column scales of a chunk as 16-byte
+    // pieces.  The row stride matters only when there is more than one chunk.
+    const bool multi_chunk = K > 128;
+    if (multi_chunk && sb_stride_kb < N) return FP8_ERR_LAYOUT;
+    if (!aligned16(sb) || (multi_chunk && sb_stride_kb % 4 != 0)) return FP8_ERR_ALIGN;
+    GemmParams out{};
+    out.c = c; out.ldc = ldc;
+    return dense_gemm<false, true>(a, lda, sa, sa_stride_m, sa_stride_kb, b, ldb, sb, sb_stride_kb,
+                                   1, out, c_type, M, N, K, stream);
 }
 
 fp8_status_t fp8_grouped_gemm(const uint8_t* a, int64_t lda, const float* sa,

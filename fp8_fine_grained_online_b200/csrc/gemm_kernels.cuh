@@ -252,6 +252,25 @@ __device__ __forceinline__ TileCoord decode_tile(int t, const GemmParams& p,
 }
 
 // acc[kOff .. kOff+32) += s * P (32 FP32 partials from TMEM), packed FMAs.
+// Per-column B scales: acc[i] += (sa * sb[i]) * P[i] for 32 columns, sb[]
+// read from shared memory (the same four values for every lane: broadcast).
+template <int kOff>
+__device__ __forceinline__ void promote32_cols(float (&acc)[128], const uint32_t (&part)[32],
+                                               uint64_t sa2, const float* sbk) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) {
+        const float4 b = lds_f4(sbk + kOff + i);
+        const uint64_t s01 = f2_mul(sa2, f2_pack(b.x, b.y));
+        const uint64_t s23 = f2_mul(sa2, f2_pack(b.z, b.w));
+        const uint64_t d01 = f2_fma(f2_pack(__uint_as_float(part[i]), __uint_as_float(part[i + 1])),
+                                    s01, f2_pack(acc[kOff + i], acc[kOff + i + 1]));
+        const uint64_t d23 = f2_fma(f2_pack(__uint_as_float(part[i + 2]), __uint_as_float(part[i + 3])),
+                                    s23, f2_pack(acc[kOff + i + 2], acc[kOff + i + 3]));
+        f2_unpack(d01, acc[kOff + i], acc[kOff + i + 1]);
+        f2_unpack(d23, acc[kOff + i + 2], acc[kOff + i + 3]);
+    }
+}
+
 template <int kOff>
 __device__ __forceinline__ void promote32(float (&acc)[128], const uint32_t (&part)[32], float s) {
 #pragma unroll
@@ -319,25 +338,39 @@ __device__ __forceinline__ void store_row_quantized(const GemmParams& p, const f
     p.sc[row * p.sc_sm + (col0 / 128) * p.sc_snb] = s;
 }
 
-template <bool kOutBf16, bool kQuantOut = false, typename Release>
+//
+// kColScaleB: B carries one scale per row n of B (column of C) and K chunk,
+// sb[kb * sb_skb + n] (n contiguous): acc += sa[row, kb] * sb[kb, n] * P_kb.
+// The warp stages the 128 sb values of its columns for chunk kb + 1 in
+// `sb_stage` ([2][128] floats of this warp) by cp.async while it promotes
+// chunk kb.
+template <bool kOutBf16, bool kQuantOut = false, bool kColScaleB = false, typename Release>
 __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, uint64_t* tfull,
                                               volatile int* abort_flag, uint32_t tmem_base,
                                               uint32_t t_lane, int h, int lane, int64_t row,
                                               bool row_ok, int64_t col0, bool col_ok, int g,
-                                              uint32_t& chunk, Release release) {
+                                              uint32_t& chunk, Release release,
+                                              float* sb_stage = nullptr) {
     const int nkb = p.nkb;
     const float* sa_row = p.sa + (row_ok ? row : 0) * p.sa_sm;
-    const float* sb_col = p.sb + g * p.sb_sg + (col_ok ? col0 / 128 : 0) * p.sb_snb;
+    const float* sb_col = kColScaleB ? p.sb + (col_ok ? col0 : 0) + 4 * lane
+                                     : p.sb + g * p.sb_sg + (col_ok ? col0 / 128 : 0) * p.sb_snb;
+    if constexpr (kColScaleB) {
+        // The previous tile's lanes are done with both staging buffers.
+        __syncwarp();
+        if (col_ok && nkb > 0) cp_async_16(sb_stage + 4 * lane, sb_col);
+        cp_async_commit();
+    }
 
     float acc[128];
 #pragma unroll
     for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
     float sa_next = (row_ok && nkb > 0) ? __ldg(sa_row) : 0.0f;
-    float sb_next = (col_ok && nkb > 0) ? __ldg(sb_col) : 0.0f;
+    float sb_next = (!kColScaleB && col_ok && nkb > 0) ? __ldg(sb_col) : 0.0f;
 
     // Scales two chunks ahead (the loads are L2 round trips).
     float sa1 = (row_ok && nkb > 1) ? __ldg(sa_row + p.sa_skb) : 0.0f;
-    float sb1 = (col_ok && nkb > 1) ? __ldg(sb_col + p.sb_skb) : 0.0f;
+    float sb1 = (!kColScaleB && col_ok && nkb > 1) ? __ldg(sb_col + p.sb_skb) : 0.0f;
 
     // Per chunk: two round trips of 64 columns through 64 staging registers;
     // the second pair of loads is issued while the first is promoted, and the
@@ -346,27 +379,44 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, uint64_t* tfu
     uint32_t pa[32], pb[32];
     for (int kb = 0; kb < nkb; ++kb) {
         const float scale = sa_next * sb_next;
+        const uint64_t sa2p = f2_pack(sa_next, sa_next);
         float sa2 = 0.0f, sb2 = 0.0f;
         if (kb + 2 < nkb) {
             sa2 = row_ok ? __ldg(sa_row + (kb + 2) * p.sa_skb) : 0.0f;
-            sb2 = col_ok ? __ldg(sb_col + (kb + 2) * p.sb_skb) : 0.0f;
+            sb2 = (!kColScaleB && col_ok) ? __ldg(sb_col + (kb + 2) * p.sb_skb) : 0.0f;
         }
         sa_next = sa1;
         sb_next = sb1;
         sa1 = sa2;
         sb1 = sb2;
+        const float* sbk = sb_stage + (kb & 1) * 128;
+        if constexpr (kColScaleB) {
+            // Chunk kb's column scales have landed (for every lane after the
+            // warp barrier); the other buffer, read during chunk kb - 1, takes
+            // chunk kb + 1's.
+            cp_async_wait_all();
+            __syncwarp();
+            if (col_ok && kb + 1 < nkb)
+                cp_async_16(sb_stage + ((kb + 1) & 1) * 128 + 4 * lane, sb_col + (kb + 1) * p.sb_skb);
+            cp_async_commit();
+        }
 
         const uint32_t buf = chunk & 1u;
-        if (!bounded_wait(&tfull[buf], (chunk >> 1) & 1u, abort_flag)) return false;
+        if (!bounded_wait(&tfull[buf], (chunk >> 1) & 1u, abort_flag)) {
+            if constexpr (kColScaleB) cp_async_wait_all();
+            return false;
+        }
         tc_fence_after();
         const uint32_t taddr = tmem_base + t_lane + buf * kBN + h * 128;
         tmem_ld_32x32b_x32(taddr, pa);
         tmem_ld_32x32b_x32(taddr + 32, pb);
         tmem_wait_ld_dep(pa);
         tmem_wait_ld_dep(pb);
-        promote32<0>(acc, pa, scale);
+        if constexpr (kColScaleB) promote32_cols<0>(acc, pa, sa2p, sbk);
+        else promote32<0>(acc, pa, scale);
         tmem_ld_32x32b_x32(taddr + 64, pa);
-        promote32<32>(acc, pb, scale);
+        if constexpr (kColScaleB) promote32_cols<32>(acc, pb, sa2p, sbk);
+        else promote32<32>(acc, pb, scale);
         tmem_ld_32x32b_x32(taddr + 96, pb);
         tmem_wait_ld_dep(pa);
         tmem_wait_ld_dep(pb);
@@ -376,8 +426,13 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, uint64_t* tfu
         __syncwarp();
         if (lane == 0) release(buf);
         ++chunk;
-        promote32<64>(acc, pa, scale);
-        promote32<96>(acc, pb, scale);
+        if constexpr (kColScaleB) {
+            promote32_cols<64>(acc, pa, sa2p, sbk);
+            promote32_cols<96>(acc, pb, sa2p, sbk);
+        } else {
+            promote32<64>(acc, pa, scale);
+            promote32<96>(acc, pb, scale);
+        }
     }
     if (row_ok && col_ok) {
         if (kQuantOut) {

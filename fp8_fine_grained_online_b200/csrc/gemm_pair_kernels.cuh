@@ -24,6 +24,10 @@
 //
 // Per SM and chunk this moves 32 KB from L2 instead of 48 KB for a
 // 128 x 256 single-CTA tile of the same MMA time.
+//
+// kColScaleB (dense): B has one scale per row and K chunk (1x128 tiles
+// along K, the weight-gradient product's second operand) instead of one
+// per 128 x 128 block.
 #pragma once
 
 #include "gemm_kernels.cuh"
@@ -51,6 +55,11 @@ constexpr size_t kGemmPairSmemBytes =
     1024 /* alignment slack */ + kPairStages * kPairStageBytes + sizeof(GemmPairSmemTail);
 // The grouped form adds its tile table (GroupTables) after the tail.
 constexpr size_t kGemmPairGroupedSmemBytes = kGemmPairSmemBytes + sizeof(GroupTables);
+// Per-column B scales: each epilogue warp's two staging rows of 128 sb
+// values after the tail (16-byte cp.async destinations).
+constexpr size_t kGemmPairColScaleSmemBytes =
+    kGemmPairSmemBytes + kEpiWarps * 2 * 128 * sizeof(float);
+static_assert(sizeof(GemmPairSmemTail) % 16 == 0, "staging rows must be 16-byte aligned");
 
 __device__ __forceinline__ void spin_ns(uint64_t ns) {
     const uint64_t t0 = globaltimer_ns();
@@ -58,16 +67,18 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
     }
 }
 
-template <bool kGrouped, bool kOutBf16, bool kQuantOut = false>
+template <bool kGrouped, bool kOutBf16, bool kQuantOut = false, bool kColScaleB = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     blockscaled_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                                  const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
+    static_assert(!(kColScaleB && (kGrouped || kQuantOut)), "per-column B scales: dense, C only");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
     GemmPairSmemTail* tail =
         reinterpret_cast<GemmPairSmemTail*>(smem + kPairStages * kPairStageBytes);
     GroupTables* gt = reinterpret_cast<GroupTables*>(tail + 1);   // grouped only
+    float* sb_stages = reinterpret_cast<float*>(tail + 1);         // per-column sb only
     volatile int* abort_flag = &tail->abort_flag;
     auto stage_a = [&](int s) { return smem + s * kPairStageBytes; };
     auto stage_b = [&](int s) { return smem + s * kPairStageBytes + kPairHalfBytes; };
@@ -223,9 +234,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const bool row_ok = row < tc.row_end;
             const int64_t col0 = tc.n0 + h * 128;
             const bool col_ok = col0 < p.N;
-            ok = epilogue_tile<kOutBf16, kQuantOut>(
+            ok = epilogue_tile<kOutBf16, kQuantOut, kColScaleB>(
                 p, tail->tfull, abort_flag, tmem_base, t_lane, h, lane, row, row_ok, col0, col_ok,
-                tc.g, chunk, [&](uint32_t buf) { mbar_arrive_cluster(tempty_leader[buf]); });
+                tc.g, chunk, [&](uint32_t buf) { mbar_arrive_cluster(tempty_leader[buf]); },
+                sb_stages + warp * 2 * 128);
         }
         if (!ok) aborted = true;
     }

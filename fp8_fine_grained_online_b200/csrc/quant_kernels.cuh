@@ -215,6 +215,27 @@ __device__ __forceinline__ uint2 encode8_corrected(const uint64_t (&n)[4], uint6
     return out;
 }
 
+// As encode8_corrected with a scale per pair of values: s2[k] and neg_r2[k]
+// pack the scales of values 2k and 2k+1 (per-column scales, 128x1 tiles).
+__device__ __forceinline__ uint2 encode8_corrected_pairs(const uint64_t (&n)[4],
+                                                         const uint64_t (&s2)[4],
+                                                         const uint64_t (&neg_r2)[4]) {
+    uint32_t c[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint64_t q0 = f2_mul(n[k], neg_r2[k]);
+        const uint64_t t = f2_fma(q0, s2[k], n[k]);
+        const uint64_t q1 = f2_fma(t, neg_r2[k], q0);
+        float lo, hi;
+        f2_unpack(q1, lo, hi);
+        c[k] = cvt_e4m3x2(lo, hi);
+    }
+    uint2 out;
+    out.x = c[0] | (c[1] << 16);
+    out.y = c[2] | (c[3] << 16);
+    return out;
+}
+
 // Codes of 2 values through IEEE fp32 division (the definition); the
 // first value in the low byte.
 __device__ __forceinline__ uint32_t encode2_exact(float x0, float x1, float s) {

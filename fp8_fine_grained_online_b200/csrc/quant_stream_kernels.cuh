@@ -1,9 +1,13 @@
 // quant_stream_kernels.cuh -- online fine-grained E4M3 quantization streamed
-// through shared memory by TMA, in three modes:
+// through shared memory by TMA, in four modes:
 //   activations: every 1x128 tile of x [M, K] gets its own scale;
 //   weights:     every 128x128 block of w [K, N] gets its own scale, codes
 //                written [K, N] as given, or transposed to [N, K] (K
-//                contiguous, the GEMM's B operand layout).
+//                contiguous, the GEMM's B operand layout);
+//   activations along M (bf16): every 128x1 tile of x [M, K] (128 rows of
+//                one column) gets its own scale, codes written transposed
+//                to [K, M]: the 1x128 tiles of x^T that the weight gradient
+//                x^T dY contracts over.
 // scale = amax / 448 and codes E4M3_RNE_satfinite(x / scale), bit-exact to
 // IEEE fp32 division (see encode8_corrected, encode8_bracket)
 // (codingmall.com "Kan du förklara rollen för FP8 precision i
@@ -23,6 +27,7 @@
 // activations a half-warp holds 8 whole rows (8 tiles).
 #pragma once
 
+#include <cstddef>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -32,7 +37,10 @@
 
 namespace fp8fg {
 
-enum QuantMode { kQuantAct = 0, kQuantWeight = 1, kQuantWeightT = 2 };
+// kQuantActT: 128x1 activation tiles (128 consecutive rows of one column,
+// the contraction of the weight-gradient product), codes written transposed
+// [K, M] and one scale per (column, 128 rows); bf16 input only.
+enum QuantMode { kQuantAct = 0, kQuantWeight = 1, kQuantWeightT = 2, kQuantActT = 3 };
 
 constexpr int kQsGroups = 2;                 // consumer groups of 8 warps
 constexpr int kQsThreads = kQsGroups * 256;
@@ -44,7 +52,7 @@ constexpr int kQsMaxStages = 4;
 // weights.)
 template <typename T, int kMode>
 struct QsCfg {
-    static constexpr bool kTransposed = kMode == kQuantWeightT;
+    static constexpr bool kTransposed = kMode == kQuantWeightT || kMode == kQuantActT;
     static constexpr int kSlots = sizeof(T) == 2 ? 2 : 1;
     static constexpr int kStages = kQsGroups * kSlots;
     static constexpr int kBoxBytes = 128 * 128 * static_cast<int>(sizeof(T));
@@ -52,17 +60,23 @@ struct QsCfg {
     static_assert(kStages <= kQsMaxStages, "ring too long");
 };
 
-struct QsSmemTail {
+// 16-byte multiple, so that the transpose buffer after it is 16-byte aligned
+// (its column maxima are read and written as uint4).
+struct alignas(16) QsSmemTail {
     uint64_t full[kQsMaxStages];       // slot filled (TMA bytes)
     uint64_t gbar[kQsGroups];          // per-group barrier (8 warp arrivals)
     float red[kQsGroups][2][8];        // [group][block parity][warp]
     int abort_flag;
 };
 
-// [N, K] output only: [group][box parity][n][k/4 swizzled], transposed codes.
-struct QsTransposeBuf {
+// Transposed output only: [group][box parity][n][k/4 swizzled], transposed
+// codes; 128x1 tiles: per-warp column maxima [group][parity][warp][c][word].
+struct alignas(16) QsTransposeBuf {
     uint32_t tbuf[kQsGroups][2][128][33];
+    uint32_t colmax[kQsGroups][2][8][16][4];
 };
+static_assert(sizeof(QsSmemTail) % 16 == 0 && offsetof(QsTransposeBuf, colmax) % 16 == 0,
+              "uint4 access to the column maxima");
 
 template <typename T, int kMode>
 constexpr size_t quant_stream_smem_bytes() {
@@ -291,32 +305,82 @@ __global__ void __launch_bounds__(kQsThreads, 1)
             }
             continue;
         } else {
-        // One scale for the whole 128x128 box: an amax pass over the box
-        // in shared memory, a block reduction, then an encode pass.
-        float a = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            Raw8<T> r;
-            load_raw_smem<T>(row_ptr(j), c, r);
-            a = fmaxf(a, r.abs_max());
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-            a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+        constexpr bool kColScales = kMode == kQuantActT;
         const int par = static_cast<int>((i / kQsGroups) & 1);
-        if (lane == 0) tail->red[g][par][wg] = a;
-        if (!group_sync(&tail->gbar[g], gbar_uses, lane, abort_flag)) break;
-        a = tail->red[g][par][0];
+        // 128x1 tiles: one scale per column of the box, from a per-column
+        // amax (bf16 column pairs, packed maxima; NaN skipped) over the
+        // thread's 8 rows, its lane partner (the other kq of the warp) and
+        // the group's 8 warps.
+        uint64_t cs2[4], cnr2[4];     // column-pair scales (kColScales)
+        float cs[8];
+        bool col_off = false;
+        if constexpr (kColScales) {
+            uint32_t cm[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int w = 1; w < 8; ++w) a = fmaxf(a, tail->red[g][par][w]);
+            for (int j = 0; j < 8; ++j) {
+                Raw8<T> r;
+                load_raw_smem<T>(row_ptr(j), c, r);
+                cm[0] = bf16x2_max(cm[0], r.a.x & 0x7FFF7FFFu);
+                cm[1] = bf16x2_max(cm[1], r.a.y & 0x7FFF7FFFu);
+                cm[2] = bf16x2_max(cm[2], r.a.z & 0x7FFF7FFFu);
+                cm[3] = bf16x2_max(cm[3], r.a.w & 0x7FFF7FFFu);
+            }
+#pragma unroll
+            for (int w = 0; w < 4; ++w) cm[w] = bf16x2_max(cm[w], __shfl_xor_sync(0xFFFFFFFFu, cm[w], 16));
+            if (lane < 16)
+                *reinterpret_cast<uint4*>(tx->colmax[g][par][wg][c]) = make_uint4(cm[0], cm[1], cm[2], cm[3]);
+            if (!group_sync(&tail->gbar[g], gbar_uses, lane, abort_flag)) break;
+#pragma unroll
+            for (int w8 = 0; w8 < 8; ++w8) {
+                const uint4 o = *reinterpret_cast<const uint4*>(tx->colmax[g][par][w8][c]);
+                cm[0] = bf16x2_max(cm[0], o.x);
+                cm[1] = bf16x2_max(cm[1], o.y);
+                cm[2] = bf16x2_max(cm[2], o.z);
+                cm[3] = bf16x2_max(cm[3], o.w);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                cs[2 * k] = scale_from_amax(__uint_as_float(cm[k] << 16));
+                cs[2 * k + 1] = scale_from_amax(__uint_as_float(cm[k] & 0xFFFF0000u));
+                const float r0 = __frcp_rn(cs[2 * k]), r1 = __frcp_rn(cs[2 * k + 1]);
+                cs2[k] = f2_pack(cs[2 * k], cs[2 * k + 1]);
+                cnr2[k] = f2_pack(-r0, -r1);
+                col_off |= !corrected_path_ok(cs[2 * k]) || !corrected_path_ok(cs[2 * k + 1]);
+            }
+            if (kq == 0) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    p.s[(bc * 128 + c * 8 + e) * p.s_stride_r + br * p.s_stride_c] = cs[e];
+            }
+        }
+        // Otherwise one scale for the whole 128x128 box: an amax pass over
+        // the box in shared memory, a block reduction, then an encode pass.
+        float a = 0.0f;
+        if constexpr (!kColScales) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                Raw8<T> r;
+                load_raw_smem<T>(row_ptr(j), c, r);
+                a = fmaxf(a, r.abs_max());
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+                a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+            if (lane == 0) tail->red[g][par][wg] = a;
+            if (!group_sync(&tail->gbar[g], gbar_uses, lane, abort_flag)) break;
+            a = tail->red[g][par][0];
+#pragma unroll
+            for (int w = 1; w < 8; ++w) a = fmaxf(a, tail->red[g][par][w]);
+        }
         const float s = scale_from_amax(a);
         const float rcp = __frcp_rn(s);
         const float ru = rcp * kBracketUp;
         const float rd = rcp * kBracketDown;
-        const bool off_path = sizeof(T) == 2 ? !corrected_path_ok(s) : !reciprocal_path_ok(s);
+        const bool off_path = kColScales ? col_off
+                                         : (sizeof(T) == 2 ? !corrected_path_ok(s) : !reciprocal_path_ok(s));
         const uint64_t s2 = f2_pack(s, s);
         const uint64_t neg_r2 = f2_pack(-rcp, -rcp);
-        if (t == 0) p.s[br * p.s_stride_r + bc * p.s_stride_c] = s;
+        if (!kColScales && t == 0) p.s[br * p.s_stride_r + bc * p.s_stride_c] = s;
         uint32_t(*tb)[33] = tx->tbuf[g][par];
         // Word w of row n sits at column (w + 2 (n / 8)) mod 32 of a 33-word
         // row: the stores below (n = 8c + e, w = 16 h4 + kq) hit 32 distinct
@@ -337,7 +401,11 @@ __global__ void __launch_bounds__(kQsThreads, 1)
             uint32_t amb = 0;
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
-                if constexpr (sizeof(T) == 2) {
+                if constexpr (kColScales) {
+                    uint64_t n[4];
+                    raw[jj].to_neg_pairs(n);
+                    codes[jj] = encode8_corrected_pairs(n, cs2, cnr2);
+                } else if constexpr (sizeof(T) == 2) {
                     uint64_t n[4];
                     raw[jj].to_neg_pairs(n);
                     codes[jj] = encode8_corrected(n, s2, neg_r2);
@@ -355,7 +423,19 @@ __global__ void __launch_bounds__(kQsThreads, 1)
                 amb &= amb - 1;
                 float x0, x1;
                 select_pair<4>(raw, idx, x0, x1);
-                const uint32_t c16 = encode2_exact(x0, x1, s);
+                uint32_t c16;
+                if constexpr (kColScales) {   // the pair's two column scales
+                    float s0 = cs[0], s1 = cs[1];
+#pragma unroll
+                    for (int k = 1; k < 4; ++k)
+                        if ((idx & 3) == k) {
+                            s0 = cs[2 * k];
+                            s1 = cs[2 * k + 1];
+                        }
+                    c16 = cvt_e4m3x2(__fdiv_rn(x0, s0), __fdiv_rn(x1, s1));
+                } else {
+                    c16 = encode2_exact(x0, x1, s);
+                }
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj)
                     if ((idx >> 2) == jj) patch_pair(codes[jj], idx & 3, c16);
@@ -381,7 +461,7 @@ __global__ void __launch_bounds__(kQsThreads, 1)
             }
         }
         if (*abort_flag) break;
-        if (kMode == kQuantWeightT) {
+        if (kMode == kQuantWeightT || kMode == kQuantActT) {
             if (!group_sync(&tail->gbar[g], gbar_uses, lane, abort_flag)) break;
             const int n = t >> 1;
             const int part = t & 1;

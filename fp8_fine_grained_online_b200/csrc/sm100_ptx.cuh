@@ -245,6 +245,33 @@ __device__ __forceinline__ void tmem_wait_ld_dep(uint32_t (&r)[32]) {
         : "memory");
 }
 
+// 16-byte global -> shared copy that bypasses the registers (cp.async, L2
+// only), its commit and the wait for all of this thread's copies.
+__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gmem_src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                 :
+                 : "r"(smem_u32(smem_dst)), "l"(gmem_src)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+// Four fp32 values from shared memory (one 16-byte load).
+__device__ __forceinline__ float4 lds_f4(const float* p) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(smem_u32(p))
+                 : "memory");
+    return v;
+}
+
 // Two fp32 values in one 64-bit register pair (lo in the low half), and the
 // packed sm_100 FP32 operations on such pairs (each lane IEEE round-to-
 // nearest, subnormals kept).  Values stay in 64-bit registers from one

@@ -206,6 +206,61 @@ FP8FG_API fp8_status_t fp8_blockscaled_gemm_quant(const uint8_t* a, int64_t lda,
                                                   int64_t K, fp8_stream_t stream);
 
 /*
+ * fp8_quantize_act_128x1 -- 1x128 quantization of x^T, for the weight-
+ * gradient product dW = x^T dY, whose contraction runs over the M rows
+ * (tokens) of x: the activation tiles of [KB] "Finkornig kvantisering",
+ * taken along M, scaled on every call ("Online-kvantisering"), in the one
+ * E4M3 format of forward and backward ("Unified E4M3 Format"); [HS] 2.2.
+ * For every column k of x [M, K] and every 128 rows mb:
+ *     amax           = max_m |x[m, k]|          (m in [128 mb, 128 mb + 128))
+ *     st[k, mb]      = amax / 448   (1 if that is 0)
+ *     qt[k, m]       = E4M3_RNE_satfinite(x[m, k] / st[k, mb])
+ * i.e. fp8_quantize_act_1x128 of the transposed matrix, written [K, M].
+ *
+ *  x      device bf16 [M, ldx]; 16-byte aligned, ldx * 2 % 16 == 0, ldx >= K.
+ *         fp32 input: FP8_ERR_DTYPE.
+ *  qt     device codes [K, ldq]; 16-byte aligned, ldq % 16 == 0, ldq >= M.
+ *  st     device fp32, st[k * st_stride_k + mb * st_stride_mb] for
+ *         0 <= mb < M/128 (e.g. [K, M/128]: st_stride_k = M/128,
+ *         st_stride_mb = 1, the layout of sa for fp8_blockscaled_gemm_colscale;
+ *         or [M/128, K]: st_stride_k = 1, st_stride_mb = K, its sb layout).
+ *  M, K   multiples of 128 (else FP8_ERR_SHAPE); 0 is a no-op.
+ *  NaN inputs are skipped by amax and encode to the NaN code.
+ */
+FP8FG_API fp8_status_t fp8_quantize_act_128x1(const void* x, fp8_in_t x_type, int64_t M, int64_t K,
+                                              int64_t ldx, uint8_t* qt, int64_t ldq, float* st,
+                                              int64_t st_stride_k, int64_t st_stride_mb,
+                                              fp8_stream_t stream);
+
+/*
+ * fp8_blockscaled_gemm_colscale -- the block-scaled GEMM with 1x128 tiles
+ * on BOTH operands, as the weight gradient needs (both x^T and dY^T are
+ * quantized along the tokens, fp8_quantize_act_128x1): B has one scale
+ * per row n and 128-wide K chunk instead of one per 128 x 128 block.  Each
+ * chunk's tensor-core partial is promoted into FP32 with the scale
+ * products ([KB] "Ökad ackumuleringsprecision"):
+ *
+ *     C[m, n] = sum_kb sa[m, kb] * sb[kb, n] * P_kb[m, n]
+ *
+ *  a, sa  as in fp8_blockscaled_gemm ([M, lda] codes, sa[m * sa_stride_m +
+ *         kb * sa_stride_kb]).
+ *  b      device codes [N, ldb], K contiguous; alignment as a.
+ *  sb     device fp32 [K/128, sb_stride_kb]: sb[kb * sb_stride_kb + n], n
+ *         contiguous; 16-byte aligned; when K > 128 also
+ *         sb_stride_kb % 4 == 0 and sb_stride_kb >= N (one chunk: any
+ *         stride).
+ *  c      device [M, ldc] of c_type; as fp8_blockscaled_gemm.
+ *  M >= 0 any value; N and K multiples of 128; K == 0 writes C = 0.
+ *  Errors: as fp8_blockscaled_gemm.
+ */
+FP8FG_API fp8_status_t fp8_blockscaled_gemm_colscale(const uint8_t* a, int64_t lda, const float* sa,
+                                                     int64_t sa_stride_m, int64_t sa_stride_kb,
+                                                     const uint8_t* b, int64_t ldb, const float* sb,
+                                                     int64_t sb_stride_kb, void* c,
+                                                     fp8_out_t c_type, int64_t ldc, int64_t M,
+                                                     int64_t N, int64_t K, fp8_stream_t stream);
+
+/*
  * fp8_grouped_gemm -- the block-scaled GEMM over MoE expert groups.
  * Same arithmetic as fp8_blockscaled_gemm ([KB] "Mixed Precision
  * Framework", "Ökad ackumuleringsprecision"), applied per expert g to the

@@ -17,7 +17,7 @@ Recipe (every tensor has its own seed, ``seed_for(config, tensor)``):
     random (the first ``topk`` of a seeded random permutation per token);
     routed rows are sorted by expert, ties in token order.
 
-The five workloads follow the DeepSeek-V3 shapes the FP8 scheme is used on
+The six workloads follow the DeepSeek-V3 shapes the FP8 scheme is used on
 (hidden 7168, FFN 18432, 256 experts with top-8 routing, expert dims
 2048 / 4096).
 """
@@ -92,7 +92,7 @@ class Workload:
     shapes: dict = field(default_factory=dict)
 
 
-# The five workloads (names are used by tests and by bench.py).
+# The six workloads (names are used by tests and by bench.py).
 TINY = Workload("tiny_e2e_128x256x256", 0,
                 "A fp32 [128x256], B fp32 [256x256], N(0,1) with 1% set to +-50; "
                 "1x128 act quant, 128x128 weight quant, block-scaled GEMM -> fp32 C",
@@ -113,7 +113,13 @@ DGRAD = Workload("dgrad_16384x7168x18432", 4,
                  "N(0,0.02); dX = dY W^T -> bf16 [16384x7168]",
                  dict(M=16384, K=18432, N=7168))
 
-WORKLOADS = {w.name: w for w in (TINY, QUANT, FFN, MOE, DGRAD)}
+WGRAD = Workload("wgrad_7168x18432_over_16384tok", 5,
+                 "X bf16 [16384x7168] N(0,1) 0.1% outliers x100, dY bf16 [16384x18432] "
+                 "N(0,1e-3) 0.1% outliers x100; dW = X^T dY -> fp32 [7168x18432], both "
+                 "operands 1x128 along the 16384 tokens",
+                 dict(M=16384, K=7168, N=18432))
+
+WORKLOADS = {w.name: w for w in (TINY, QUANT, FFN, MOE, DGRAD, WGRAD)}
 
 
 def tiny_inputs(device="cpu"):
@@ -159,6 +165,15 @@ def dgrad_inputs(device="cpu", M=16384, K=18432, N=7168):
     dy = act_input(M, K, 1e-3, 1e-3, 100.0, c, device)
     w = weight_input(N, K, 0.02, c, device)
     return dy, w
+
+
+def wgrad_inputs(device="cpu", M=16384, K=7168, N=18432):
+    """X [M, K] (the layer input) and dY [M, N] (its output gradient); the
+    weight gradient contracts over the M tokens."""
+    c = WGRAD.config_id
+    x = act_input(M, K, 1.0, 1e-3, 100.0, c, device)
+    dy = act_input(M, N, 1e-3, 1e-3, 100.0, c, device, tensor_id=2)
+    return x, dy
 
 
 def moe_inputs(device="cpu", tokens=8192, experts=256, topk=8, hidden=7168, inter=2048,

@@ -206,3 +206,40 @@ def test_gather_quant_argument_errors(L):
     assert call(ldq=64) == 4
     assert call(ldx=132) == 3          # ldx * 2 bytes % 16
     assert call(rows=vp(base + 2)) == 3
+
+
+def test_act_128x1_argument_errors(L):
+    # x, x_type, M, K, ldx, qt, ldq, st, st_k, st_mb, stream
+    def call(x=A16, xt=0, M=256, K=128, ldx=128, qt=A16, ldq=256, st=A16, sk=2, smb=1):
+        return L.fp8_quantize_act_128x1(x, xt, M, K, ldx, qt, ldq, st, sk, smb, None)
+    assert call(xt=7) == 5
+    assert call(M=200) == 2                        # M % 128 (the tile runs along M)
+    assert call(K=100, ldx=128) == 2
+    assert call(M=0, x=None, qt=None, st=None) == 0
+    assert call(xt=1) == 5                         # bf16 input only
+    assert call(qt=None) == 1
+    assert call(ldq=128) == 4                      # qt is [K, M]: ldq >= M
+    assert call(ldx=64) == 4
+    assert call(smb=-1) == 4
+    assert call(x=A8) == 3
+    assert call(ldq=264) == 3
+    assert call(st=P(0x10002)) == 3
+
+
+def test_gemm_colscale_argument_errors(L):
+    # a, lda, sa, sa_m, sa_kb, b, ldb, sb, sb_kb, c, c_type, ldc, M, N, K, stream
+    def call(a=A16, sa=A16, b=A16, sb=A16, sbkb=256, c=A16, ct=1, ldc=256, M=128, N=256,
+             K=256):
+        return L.fp8_blockscaled_gemm_colscale(a, 256, sa, 2, 1, b, 256, sb, sbkb, c, ct, ldc, M,
+                                               N, K, None)
+    assert call(ct=4) == 5
+    assert call(N=100) == 2
+    assert call(K=200) == 2
+    assert call(M=0, a=None) == 0
+    assert call(sb=None) == 1
+    assert call(sbkb=128) == 4                     # sb rows hold N values
+    assert call(sbkb=258) == 3                     # 16-byte pieces of a row: stride % 4
+    if not __import__("torch").cuda.is_available():
+        assert call(sbkb=1, K=128) == 6            # one chunk: the row stride is unused
+    assert call(sb=P(0x10004)) == 3
+    assert call(ldc=260) == 3
