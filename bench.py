@@ -203,6 +203,41 @@ class Workload:
         """Units of `value` per step (FLOP or bytes)."""
         raise NotImplementedError
 
+    def e2e_teardown(self):
+        """Drop the pinned host copies made by e2e_setup."""
+        for k in list(vars(self)):
+            v = getattr(self, k)
+            if isinstance(v, torch.Tensor) and not v.is_cuda and k.startswith("h"):
+                delattr(self, k)
+
+
+def error_vs_exact(c, exact, sample):
+    """Quantization error of the FP8 path against the unquantized product,
+    both fp64 tensors of the same sampled entries: max|C - E| / max|E| and
+    the relative Frobenius error ||C - E|| / ||E||."""
+    d = c - exact
+    return {"max_rel": float(d.abs().max() / exact.abs().max()),
+            "fro_rel": float(torch.linalg.norm(d) / torch.linalg.norm(exact)),
+            "entries": int(exact.numel()), "sample": sample}
+
+
+def sample_index(n, count, device):
+    """`count` indices spread evenly over range(n) (all of them if n <= count)."""
+    count = min(n, count)
+    return (torch.arange(count, device=device, dtype=torch.int64) * n) // count
+
+
+def quant_error_tiny(fp8, device):
+    """The tiny end-to-end config in full: A fp32 [128x256], B fp32 [256x256]
+    quantized (1x128 / 128x128), block-scaled GEMM -> fp32, against the fp64
+    product of the unquantized A and B."""
+    a, b = synth.tiny_inputs(device)
+    qa, sa = fp8.fp8_quantize_act_1x128(a)
+    qb, sb = fp8.fp8_quantize_weight_128x128(b, transpose_out=True)
+    c = fp8.fp8_blockscaled_gemm(qa, sa, qb, sb, out_dtype=torch.float32)
+    exact = a.double() @ b.double()
+    return error_vs_exact(c.double(), exact, "all 128 x 256 entries")
+
 
 class FFN(Workload):
     """Online-quantized dense FFN up-projection forward."""
@@ -254,6 +289,17 @@ class FFN(Workload):
         f.fp8_blockscaled_gemm(self.qx, self.sx, self.qw, self.sw, c=self.c)
         marks(3)
 
+    def quant_error(self, rows=256, blocks=16):
+        """Last step's bf16 C on a spread sample of rows x 128-column blocks
+        against the fp64 product of the unquantized bf16 X and W."""
+        dev = self.c.device
+        r = sample_index(self.M, rows, dev)
+        nb = sample_index(self.N // 128, blocks, dev)
+        cols = (nb[:, None] * 128 + torch.arange(128, device=dev)).reshape(-1)
+        exact = self.x[r].double() @ self.w[:, cols].double()
+        return error_vs_exact(self.c[r][:, cols].double(), exact,
+                              "%d rows x %d 128-column blocks, spread evenly" % (len(r), len(nb)))
+
     # end to end through the public API with pinned host buffers
     def e2e_setup(self):
         self.hx = self.x.cpu().pin_memory()
@@ -303,6 +349,8 @@ class FFNQuantOut(FFN):
         d["workload"] = self.name
         d["out"] = "E4M3 [%dx%d] + fp32 1x128 scales (quantized in the GEMM epilogue)" % (self.M, self.N)
         return d
+
+    quant_error = None     # no bf16 C is kept (the ffn workload reports it)
 
     def algorithmic(self):
         d = super().algorithmic()
@@ -516,6 +564,17 @@ class DGrad(FFN):
             "blockscaled_gemm": ("flops", 2.0 * M * N * K),
         }
 
+    def quant_error(self, rows=256, blocks=16):
+        """dX = dY W^T on a sample of rows x 128-column blocks against the fp64
+        product of the unquantized bf16 dY and W."""
+        dev = self.c.device
+        r = sample_index(self.M, rows, dev)
+        nb = sample_index(self.N // 128, blocks, dev)
+        cols = (nb[:, None] * 128 + torch.arange(128, device=dev)).reshape(-1)
+        exact = self.x[r].double() @ self.w[cols].double().t()
+        return error_vs_exact(self.c[r][:, cols].double(), exact,
+                              "%d rows x %d 128-column blocks, spread evenly" % (len(r), len(nb)))
+
     def step(self, marks):
         f = self.fp8
         marks(0)
@@ -599,6 +658,17 @@ class WGrad(Workload):
             "blockscaled_gemm_colscale": ("flops", 2.0 * M * N * K),
         }
 
+    def quant_error(self, rows=256, blocks=16):
+        """dW = X^T dY on a sample of rows x 128-column blocks against the fp64
+        product of the unquantized bf16 X and dY (contraction over all tokens)."""
+        dev = self.c.device
+        r = sample_index(self.K, rows, dev)
+        nb = sample_index(self.N // 128, blocks, dev)
+        cols = (nb[:, None] * 128 + torch.arange(128, device=dev)).reshape(-1)
+        exact = self.x[:, r].double().t() @ self.dy[:, cols].double()
+        return error_vs_exact(self.c[r][:, cols].double(), exact,
+                              "%d rows x %d 128-column blocks, spread evenly" % (len(r), len(nb)))
+
     def step(self, marks):
         f = self.fp8
         marks(0)
@@ -647,15 +717,17 @@ class MoE(Workload):
         self.fp8 = fp8
         self.T, self.E, self.k, self.H, self.I = tokens, experts, topk, hidden, inter
         self.R = tokens * topk
-        self.kernels = ["quant_act_1x128_gather_x", "grouped_gemm_gate_up", "quant_act_1x128_h",
+        self.kernels = ["quant_act_1x128_scatter_x", "grouped_gemm_gate_up", "quant_act_1x128_h",
                         "grouped_gemm_down"]
         if device is None:
             return
         d = synth.moe_inputs(device, tokens, experts, topk, hidden, inter, with_weights=False)
-        # tokens and their routing: the dispatch (row gather by expert) is
+        # tokens and their routing: the dispatch (token rows to expert order) is
         # fused into the activation quantizer
         self.x, self.h, self.off = d["x"], d["h_down"], d["offsets"]
         self.rows = d["token_of"].to(torch.int32)
+        # the same routing in token order: token t's topk expert-sorted rows
+        self.dest = synth.moe_dispatch_dest(d["token_of"], tokens, topk)
         del d
         R, H, I, E = self.R, hidden, inter, experts
         self.qgu = torch.empty((E, 2 * I, H), dtype=torch.uint8, device=device)
@@ -681,14 +753,15 @@ class MoE(Workload):
                 "routed_rows": self.R, "gate_up": "K=%d N=%d" % (self.H, 2 * self.I),
                 "down": "K=%d N=%d" % (self.I, self.H), "out": "bf16",
                 "weights": "quantized once before timing (11.27 GB E4M3)",
-                "dispatch": "token rows gathered by expert inside the activation quantizer",
+                "dispatch": "each token row quantized once inside the activation quantizer and "
+                            "written to its 8 expert-sorted rows",
                 "l2": "expert weights 11.27 GB >> L2"}
 
     def algorithmic(self):
         R, H, I, E = self.R, self.H, self.I, self.E
         return {
             # tokens read once, routed rows written (codes + scales)
-            "quant_act_1x128_gather_x": ("bytes", self.T * H * 2 + R * H + R * (H // 128) * 4),
+            "quant_act_1x128_scatter_x": ("bytes", self.T * H * 2 + R * H + R * (H // 128) * 4),
             "grouped_gemm_gate_up": ("flops", 2.0 * R * 2 * I * H),
             "quant_act_1x128_h": ("bytes", R * I * 3 + R * (I // 128) * 4),
             "grouped_gemm_down": ("flops", 2.0 * R * H * I),
@@ -708,7 +781,7 @@ class MoE(Workload):
     def step(self, marks):
         f = self.fp8
         marks(0)
-        f.fp8_quantize_act_1x128_gather(self.x, self.rows, q=self.qx, sa=self.sx)
+        f.fp8_quantize_act_1x128_scatter(self.x, self.dest, self.R, q=self.qx, sa=self.sx)
         marks(1)
         f.fp8_grouped_gemm(self.qx, self.sx, self.qgu, self.sgu, self.off, c=self.cgu)
         marks(2)
@@ -719,21 +792,21 @@ class MoE(Workload):
 
     def e2e_setup(self):
         self.hx = self.x.cpu().pin_memory()
-        self.hrows = self.rows.cpu().pin_memory()
+        self.hdest = self.dest.cpu().pin_memory()
         self.hh = self.h.cpu().pin_memory()
         self.hoff = self.off.cpu().pin_memory()
         self.hgu = torch.empty_like(self.cgu, device="cpu").pin_memory()
         self.hdn = torch.empty_like(self.cdn, device="cpu").pin_memory()
-        return ((self.hx.numel() + self.hh.numel()) * 2 + (self.hoff.numel() + self.hrows.numel()) * 4,
+        return ((self.hx.numel() + self.hh.numel()) * 2 + (self.hoff.numel() + self.hdest.numel()) * 4,
                 (self.hgu.numel() + self.hdn.numel()) * 2)
 
     def e2e_step(self):
         f = self.fp8
         x = self.hx.to("cuda", non_blocking=True)
-        rows = self.hrows.to("cuda", non_blocking=True)
+        dest = self.hdest.to("cuda", non_blocking=True)
         h = self.hh.to("cuda", non_blocking=True)
         off = self.hoff.to("cuda", non_blocking=True)
-        qx, sx = f.fp8_quantize_act_1x128_gather(x, rows)
+        qx, sx = f.fp8_quantize_act_1x128_scatter(x, dest, self.R)
         cgu = f.fp8_grouped_gemm(qx, sx, self.qgu, self.sgu, off)
         qh, sh = f.fp8_quantize_act_1x128(h)
         cdn = f.fp8_grouped_gemm(qh, sh, self.qdn, self.sdn, off)
@@ -762,9 +835,14 @@ class MoE(Workload):
 
 WORKLOADS = {"ffn": FFN, "ffn_q": FFNQuantOut, "quant": Quant, "moe": MoE, "dgrad": DGrad,
              "dequant": Dequant, "wgrad": WGrad}
-# Oracle sample per step: (rows, column blocks), sized for a few seconds per step.
-ORACLE_SAMPLE = {"ffn": (32, 2), "ffn_q": (32, 2), "quant": (16, 4), "moe": (32, 1), "dgrad": (16, 1),
-                 "dequant": (64, 8), "wgrad": (16, 1)}
+# Reported with the default run, after the FFN headline, each in its own timed region.
+EXTRA_WORKLOADS = ("quant", "dgrad", "wgrad", "moe", "ffn_q", "dequant")
+# Oracle sample per step of the reference arm: (rows, column blocks).  Each is
+# about 60% of the CPU-baseline sample below, with the same balance of
+# quantization and GEMM work (so that both arms measure the oracle alike),
+# and a 25-step run stays within a few minutes.
+ORACLE_SAMPLE = {"ffn": (768, 32), "ffn_q": (768, 32), "quant": (256, 144), "moe": (256, 24),
+                 "dgrad": (256, 14), "dequant": (512, 144), "wgrad": (256, 24)}
 # The single CPU-baseline measurement of a run: about 10 s of oracle work.
 CPU_BASELINE_SAMPLE = {"ffn": (1024, 60), "ffn_q": (1024, 60), "quant": (512, 144),
                        "moe": (512, 24), "dgrad": (256, 24), "dequant": (896, 144),
@@ -799,11 +877,12 @@ def make_workload(args, fp8, device):
     return WORKLOADS[args.workload](fp8, device)
 
 
-def run_ours(args, rank, world, local_rank):
-    import fp8_fine_grained_online_b200 as fp8
-    device = "cuda:%d" % local_rank
-    torch.cuda.set_device(local_rank)
-    wl = make_workload(args, fp8, device)
+def time_workload(wl, args, world, device, fp8):
+    """W untimed warm-up steps, then exactly K steps between barriers and
+    device synchronizations, timed with CUDA events on the launching stream
+    (whole region and each kernel of each step); SM clocks sampled during the
+    timed region.  Returns (max-over-ranks ms, per-kernel mean ms, clocks,
+    wall seconds, device error word)."""
     stream = torch.cuda.current_stream()
     nk = len(wl.kernels)
 
@@ -815,7 +894,7 @@ def run_ours(args, rank, world, local_rank):
         wl.step(lambda i: None)
     torch.cuda.synchronize()
     if fp8.fp8_get_device_error() != 0:
-        raise RuntimeError("device error during warm-up")
+        raise RuntimeError("device error during warm-up of %s" % wl.name)
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -835,11 +914,25 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     elapsed_ms = max_over_ranks(start.elapsed_time(stop), world, device)
     dev_err = fp8.fp8_get_device_error()
-
     per_kernel = {}
     for i, k in enumerate(wl.kernels):
         per_kernel[k] = statistics.fmean(ev[s][i].elapsed_time(ev[s][i + 1])
                                          for s in range(args.steps))
+    return elapsed_ms, per_kernel, clk, wall, dev_err
+
+
+def run_ours(args, rank, world, local_rank):
+    import fp8_fine_grained_online_b200 as fp8
+    device = "cuda:%d" % local_rank
+    torch.cuda.set_device(local_rank)
+    wl = make_workload(args, fp8, device)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    elapsed_ms, per_kernel, clk, wall, dev_err = time_workload(wl, args, world, device, fp8)
 
     # end to end through the public API, pinned host buffers
     e2e = None
@@ -860,7 +953,40 @@ def run_ours(args, rank, world, local_rank):
         e2e = {"value": round(aggregate_rate(world, wl.work_per_step(), n_e2e, e_ms) / scale(wl), 3),
                "unit": wl.unit, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": n_e2e}
+        wl.e2e_teardown()
     return wl, elapsed_ms, per_kernel, clk, e2e, wall, dev_err
+
+
+def run_extra(args, name, world, local_rank, peaks, peak_src):
+    """One more workload on the same process (every rank, as for the
+    headline): its own timed region, kernels, roofline and clocks."""
+    import fp8_fine_grained_online_b200 as fp8
+    device = "cuda:%d" % local_rank
+    wl = WORKLOADS[name](fp8, device)
+    elapsed_ms, per_kernel, clk, wall, dev_err = time_workload(wl, args, world, device, fp8)
+    rec = workload_record(wl, name, world, args, elapsed_ms, per_kernel, peaks, peak_src)
+    rec.update({"clocks": clk, "device_error": dev_err, "wall_s_timed_region": round(wall, 4)})
+    err = wl.quant_error() if callable(getattr(wl, "quant_error", None)) else None
+    del wl
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec, err
+
+
+def workload_record(wl, name, world, args, elapsed_ms, per_kernel, peaks, peak_src):
+    value = aggregate_rate(world, wl.work_per_step(), args.steps, elapsed_ms) / scale(wl)
+    kernels = {}
+    for k, ms in per_kernel.items():
+        r = roofline_entry(wl, k, ms, peaks, peak_src)
+        kernels[k] = {"us": round(ms * 1e3, 2), "achieved": r["achieved"], "unit": r["unit"],
+                      "frac": r["frac"], "bound": r["bound"],
+                      "traffic": recorded_traffic(k, name)}
+    roof = roofline_entry(wl, wl.dominant, per_kernel[wl.dominant], peaks, peak_src)
+    roof["traffic"] = recorded_traffic(wl.dominant, name)
+    return {"config": wl.config(), "value": round(value, 3), "unit": wl.unit,
+            "ms_per_step": round(elapsed_ms / args.steps, 4), "steps": args.steps,
+            "warmup": args.warmup, "gpu_launches": len(wl.kernels) * args.steps,
+            "roofline": roof, "kernels": kernels}
 
 
 def scale(wl):
@@ -914,6 +1040,10 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="ffn")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--extra", default=None,
+                    help="comma list of workloads timed after the headline and reported under "
+                         "'workloads' (default: all others when the headline is ffn; 'none')")
+    ap.add_argument("--no-quant-error", action="store_true")
     ap.add_argument("--moe-experts", type=int, default=256,
                     help="MoE workload only: number of experts (tokens = 32 x experts)")
     args = ap.parse_args()
@@ -958,33 +1088,56 @@ def main():
     if world > 1:
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
+    extras = parse_extra(args)
     try:
+        import fp8_fine_grained_online_b200 as fp8
         wl, elapsed_ms, per_kernel, clk, e2e, wall, dev_err = run_ours(args, rank, world,
                                                                        local_rank)
+        peaks, peak_src = load_peaks()
+        # Quantization error of the FP8 path against the unquantized fp64
+        # product: the tiny config in full, the headline on a sample.
+        errors = {}
+        if not args.no_quant_error:
+            errors["tiny"] = quant_error_tiny(fp8, "cuda:%d" % local_rank)
+            if callable(getattr(wl, "quant_error", None)):
+                errors[args.workload] = wl.quant_error()
+        head = workload_record(wl, args.workload, world, args, elapsed_ms, per_kernel, peaks,
+                               peak_src)
+        del wl
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        # The other configurations, each timed in its own region like the
+        # headline (its own warm-up, steps, clocks and roofline).
+        others = {}
+        for name in extras:
+            rec, err = run_extra(args, name, world, local_rank, peaks, peak_src)
+            others[name] = rec
+            if err is not None and not args.no_quant_error:
+                errors[name] = err
         if rank != 0:
             return
-        peaks, peak_src = load_peaks()
-        value = aggregate_rate(world, wl.work_per_step(), args.steps, elapsed_ms) / scale(wl)
-        kernels = {}
-        for k, ms in per_kernel.items():
-            r = roofline_entry(wl, k, ms, peaks, peak_src)
-            kernels[k] = {"us": round(ms * 1e3, 2), "achieved": r["achieved"], "unit": r["unit"],
-                          "frac": r["frac"]}
-        dom = wl.dominant
-        roof = roofline_entry(wl, dom, per_kernel[dom], peaks, peak_src)
-        roof["traffic"] = recorded_traffic(dom, args.workload)
         line = {
-            "metric": METRIC, "value": round(value, 3), "unit": wl.unit, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(elapsed_ms / args.steps, 4), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate)",
-            "data": "synthetic (seeded, DeepSeek-V3 layer shapes)", "config": wl.config(),
-            "roofline": roof, "kernels": kernels,
-            "gpu_launches": len(wl.kernels) * args.steps,
+            "metric": METRIC, "value": head["value"], "unit": head["unit"], "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3 (fp32 accumulate)",
+            "data": "synthetic (seeded, DeepSeek-V3 layer shapes)", "config": head["config"],
+            "roofline": head["roofline"], "kernels": head["kernels"],
+            "gpu_launches": head["gpu_launches"],
             "clocks": clk, "e2e": e2e, "device_error": dev_err,
             "wall_s_timed_region": round(wall, 4),
             "parallelism": "replicas (dp%d, no collective on the data path)" % world,
+            "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"],
+                      "source": peak_src},
         }
+        if errors:
+            line["quant_error"] = {
+                "reference": "fp64 product of the unquantized inputs (C_exact)",
+                "metrics": "max_rel = max|C - C_exact| / max|C_exact|; "
+                           "fro_rel = ||C - C_exact||_F / ||C_exact||_F",
+                **errors}
+        if others:
+            line["workloads"] = others
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(args, wl_cls)
         print(json.dumps(line))
@@ -992,6 +1145,19 @@ def main():
         if world > 1:
             torch.distributed.destroy_process_group()
 
+
+def parse_extra(args):
+    """Workloads timed after the headline: by default every other
+    configuration when the headline is the FFN forward, none otherwise."""
+    if args.extra is None:
+        return list(EXTRA_WORKLOADS) if args.workload == "ffn" else []
+    if args.extra == "none":
+        return []
+    names = [n for n in args.extra.split(",") if n]
+    for n in names:
+        if n not in WORKLOADS:
+            raise SystemExit("unknown workload in --extra: %s" % n)
+    return [n for n in names if n != args.workload]
 
 if __name__ == "__main__":
     main()

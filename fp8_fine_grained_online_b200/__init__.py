@@ -27,8 +27,9 @@ __all__ = [
     "fp8_quantize_act_1x128", "fp8_quantize_weight_128x128", "fp8_blockscaled_gemm",
     "fp8_grouped_gemm", "fp8_status_string", "fp8_get_device_error", "Fp8Error",
     "LIB_PATH", "linear_forward", "e2e_linear_forward", "fp8_quantize_act_1x128_gather",
+    "fp8_quantize_act_1x128_scatter",
     "fp8_blockscaled_gemm_quant", "fp8_dequantize", "fp8_quantize_act_128x1",
-    "fp8_blockscaled_gemm_colscale", "linear_weight_grad",
+    "fp8_blockscaled_gemm_colscale", "linear_weight_grad", "fp8_set_wait_limit",
 ]
 
 _L = _lib.lib
@@ -76,6 +77,13 @@ def fp8_get_device_error(stream=None):
     return code.value
 
 
+def fp8_set_wait_limit(cycles):
+    """Set how many SM cycles a wait in this library's kernels may last on
+    the current device before the kernel gives up (0 restores the default,
+    about one second).  For tests of the timeout path."""
+    _lib.check(_L.fp8_set_wait_limit(int(cycles)), "fp8_set_wait_limit")
+
+
 def fp8_quantize_act_1x128(x, q=None, sa=None, stream=None):
     """x [M, K] (bf16/fp32, CUDA) -> (q uint8 [M, K] E4M3 codes, sa fp32 [M, K/128])."""
     _rowmajor(x, "x")
@@ -108,6 +116,30 @@ def fp8_quantize_act_1x128_gather(x, rows, q=None, sa=None, stream=None):
                                           _ptr(q), q.stride(0), _ptr(sa), sa.stride(0),
                                           sa.stride(1), _stream(stream))
     _lib.check(st, "fp8_quantize_act_1x128_gather")
+    return q, sa
+
+
+def fp8_quantize_act_1x128_scatter(x, dest, R, q=None, sa=None, stream=None):
+    """x [T, K] (bf16, CUDA), dest int32 [T, topk] (CUDA; -1 = none) ->
+    (q uint8 [R, K], sa fp32 [R, K/128]) where every output row
+    dest[t, j] holds the 1x128 quantization of x[t].  Each token is read
+    and quantized once.  Rows that no dest entry names are left as they
+    were (uninitialised when q / sa are allocated here)."""
+    _rowmajor(x, "x")
+    T, K = x.shape
+    if dest.dtype != torch.int32 or dest.dim() != 2 or not dest.is_contiguous() \
+            or dest.shape[0] != T:
+        raise ValueError("dest must be a contiguous int32 [T, topk] tensor")
+    topk = dest.shape[1]
+    if q is None:
+        q = torch.empty((R, K), dtype=torch.uint8, device=x.device)
+    if sa is None:
+        sa = torch.empty((R, K // 128), dtype=torch.float32, device=x.device)
+    _rowmajor(q, "q")
+    st = _L.fp8_quantize_act_1x128_scatter(_ptr(x), _in_type(x), T, K, x.stride(0), _ptr(dest),
+                                           topk, _ptr(q), R, q.stride(0), _ptr(sa), sa.stride(0),
+                                           sa.stride(1), _stream(stream))
+    _lib.check(st, "fp8_quantize_act_1x128_scatter")
     return q, sa
 
 
@@ -180,7 +212,12 @@ def fp8_blockscaled_gemm_quant(a, sa, b, sb, qc=None, sc=None, c=None, want_c=Fa
 def fp8_quantize_act_128x1(x, qt=None, st=None, st_kb_major=False, stream=None):
     """x [M, K] (bf16, CUDA) -> 1x128 quantization of x^T along M:
     (qt uint8 [K, M] E4M3 codes, st fp32 scales), st [K, M/128] or, with
-    ``st_kb_major``, [M/128, K] (the layout of the column-scale GEMM's sb)."""
+    ``st_kb_major``, [M/128, K] (the layout of the column-scale GEMM's sb).
+
+    Limits of the CUDA kernel: x must be bfloat16 (float32 raises Fp8Error
+    with FP8_ERR_DTYPE) and M a multiple of 128 (a ragged token count such as
+    a per-expert MoE batch raises FP8_ERR_SHAPE; pad it with zero rows,
+    which change no scale or code of the other rows)."""
     _rowmajor(x, "x")
     M, K = x.shape
     if qt is None:
@@ -219,7 +256,9 @@ def linear_weight_grad(x, dy, out_dtype=torch.float32, stream=None):
     """Weight gradient of y = x @ w in FP8: dW [K, N] = x^T dy with x [M, K],
     dy [M, N] (bf16).  Both are quantized in 1x128 tiles along the tokens M
     (scales computed on this call), then multiplied by the column-scale GEMM.
-    Three library calls."""
+    Three library calls.  Needs bfloat16 x and dy (else FP8_ERR_DTYPE) and
+    M a multiple of 128 (else FP8_ERR_SHAPE: pad ragged token counts with
+    zero rows, which add nothing to dW)."""
     qxt, sxt = fp8_quantize_act_128x1(x, stream=stream)
     qdt, sdt = fp8_quantize_act_128x1(dy, st_kb_major=True, stream=stream)
     return fp8_blockscaled_gemm_colscale(qxt, sxt, qdt, sdt, out_dtype=out_dtype, stream=stream)

@@ -26,6 +26,8 @@ SIGNATURES = {
                                       _vp]),
     "fp8_quantize_act_1x128_gather": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _i64, _vp, _i64,
                                              _vp, _i64, _i64, _vp]),
+    "fp8_quantize_act_1x128_scatter": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _i64, _vp,
+                                              _i64, _i64, _vp, _i64, _i64, _vp]),
     "fp8_quantize_weight_128x128": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _int, _i64, _vp,
                                            _i64, _i64, _vp]),
     "fp8_blockscaled_gemm": (_int, [_vp, _i64, _vp, _i64, _i64, _vp, _i64, _int, _vp, _i64, _i64,
@@ -43,6 +45,7 @@ SIGNATURES = {
                               _vp]),
     "fp8_status_string": (ctypes.c_char_p, [_int]),
     "fp8_get_device_error": (_int, [_vp, ctypes.POINTER(_int)]),
+    "fp8_set_wait_limit": (_int, [_i64]),
 }
 
 

@@ -9,7 +9,9 @@
 // contiguous bytes and, for bf16, stores 512 as whole 32-byte sectors) and
 // kDqRowsInFlight rows at a time, all loads issued before the first is
 // used, so that enough bytes are in flight per SM to cover HBM latency.
-// Block (x, y): 2048 codes of the rows y, y + gridDim.y, ...
+// Block (x, y): 2048 codes of the rows y, y + gridDim.y, ...  The scale row
+// of code row r is r >> tile_shift (tile_shift = log2 of the tile height:
+// 0 for 1x128 tiles, 7 for 128x128 blocks).
 #pragma once
 
 #include <cstdint>
@@ -72,7 +74,7 @@ template <bool kOutBf16>
 __global__ void __launch_bounds__(kDqThreads, kDqBlocksPerSm)
     dequant_kernel(const uint8_t* __restrict__ q, int64_t rows, int64_t cols, int64_t ldq,
                    const float* __restrict__ s, int64_t s_stride_r, int64_t s_stride_c,
-                   int tile_rows, void* __restrict__ out, int64_t ldo) {
+                   int tile_shift, void* __restrict__ out, int64_t ldo) {
     const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kDqCodesPerBlock +
                        threadIdx.x * kDqCodesPerThread;
     if (c0 >= cols) return;
@@ -86,7 +88,7 @@ __global__ void __launch_bounds__(kDqThreads, kDqBlocksPerSm)
             const int64_t r = r0 + i * step;
             if (r < rows) {
                 codes[i] = __ldcs(reinterpret_cast<const uint2*>(q + r * ldq + c0));
-                sc[i] = __ldg(s_col + (r / tile_rows) * s_stride_r);
+                sc[i] = __ldg(s_col + (r >> tile_shift) * s_stride_r);
             }
         }
 #pragma unroll

@@ -18,6 +18,8 @@
 #include "quant_stream_kernels.cuh"
 #include "dequant_kernels.cuh"
 #include "quant_gather_kernels.cuh"
+#include "quant_act_kernels.cuh"
+#include "quant_weight_kernels.cuh"
 
 namespace fp8fg {
 namespace {
@@ -82,6 +84,21 @@ fp8_status_t current_device(int* dev_out, int* sms_out) {
                     if (cudaFuncSetAttribute(pair_kernels[i],
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(bytes)) != cudaSuccess) {
+                        cudaGetLastError();
+                        return FP8_ERR_CUDA;
+                    }
+                }
+                const void* qa_kernels[] = {
+                    reinterpret_cast<const void*>(&quant_act_rows_kernel<false>),
+                    reinterpret_cast<const void*>(&quant_act_rows_kernel<true>),
+                    reinterpret_cast<const void*>(&quant_weight_rows_kernel<false>),
+                    reinterpret_cast<const void*>(&quant_weight_rows_kernel<true>)};
+                const size_t qa_bytes[] = {kQaSmemBytes, kQaSmemBytes, kQwSmemBytes,
+                                           kQwSmemBytes};
+                for (int i = 0; i < 4; ++i) {
+                    if (cudaFuncSetAttribute(qa_kernels[i],
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(qa_bytes[i])) != cudaSuccess) {
                         cudaGetLastError();
                         return FP8_ERR_CUDA;
                     }
@@ -178,6 +195,7 @@ bool make_operand_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_
 }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 inline fp8_status_t launch_status() {
@@ -190,6 +208,10 @@ inline fp8_status_t launch_status() {
 // contractions amortise better (measured: K 7168 faster on the pair, K 2048
 // faster on one CTA).
 constexpr int64_t kGroupedPairMinK = 4096;
+
+// L2 bytes one raster band of the dense GEMM may hold (of the B200's 126 MB;
+// the rest serves the streamed operand's chunks and the output).
+constexpr int64_t kL2BandBytes = int64_t{72} << 20;
 
 int elem_size_in(fp8_in_t t) { return t == FP8_IN_BF16 ? 2 : (t == FP8_IN_FP32 ? 4 : 0); }
 int elem_size_out(fp8_out_t t) { return t == FP8_OUT_BF16 ? 2 : (t == FP8_OUT_FP32 ? 4 : 0); }
@@ -238,6 +260,85 @@ bool make_input_map(CUtensorMap* map, const void* base, fp8_in_t t, uint64_t row
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// bf16 activations [M, K] (row stride ld elements) for the row kernel:
+// boxes of 32 rows x 64 columns, 128-byte swizzle, zero fill out of bounds.
+bool make_act_rows_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                       uint64_t ld) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {ld * 2};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kQaRows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// 128x128 quantization of a bf16 weight [K, N], one block row per thread
+// (quant_weight_rows_kernel): boxes of 128 rows x 64 columns, 128-byte
+// swizzle; one persistent CTA of kQwGroups groups per SM.
+fp8_status_t launch_quant_weight_rows(const void* w, int64_t K, int64_t N, int64_t ldw,
+                                      uint8_t* q, int transpose_out, int64_t ldq, float* sb,
+                                      int64_t sb_stride_kb, int64_t sb_stride_nb, int sms,
+                                      cudaStream_t stream) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return FP8_ERR_CUDA;
+    CUtensorMap map;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(K)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldw) * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estr[2] = {1, 1};
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return FP8_ERR_CUDA;
+    QwParams p{};
+    p.nbr = K / 128;
+    p.nbc = N / 128;
+    p.nblocks = p.nbr * p.nbc;
+    p.q = q; p.ldq = ldq;
+    p.s = sb; p.s_stride_kb = sb_stride_kb; p.s_stride_nb = sb_stride_nb;
+    const int64_t ctas = (p.nblocks + kQwGroups - 1) / kQwGroups;
+    const unsigned grid = static_cast<unsigned>(ctas < sms ? ctas : sms);
+    if (transpose_out)
+        quant_weight_rows_kernel<true><<<grid, kQwThreads, kQwSmemBytes, stream>>>(map, p);
+    else
+        quant_weight_rows_kernel<false><<<grid, kQwThreads, kQwSmemBytes, stream>>>(map, p);
+    return launch_status();
+}
+
+// 1x128 quantization of bf16 rows, one row per thread (quant_act_rows_kernel):
+// one persistent CTA of kQaWarps independent warps per SM.
+// With `dest` (scatter form): input row t goes to the output rows
+// dest[t * topk + j] (of out_rows); otherwise row m goes to row m.
+fp8_status_t launch_quant_act_rows(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
+                                   int64_t ldq, float* sa, int64_t sa_stride_m,
+                                   int64_t sa_stride_kb, int sms, cudaStream_t stream,
+                                   const int32_t* dest = nullptr, int64_t topk = 0,
+                                   int64_t out_rows = 0) {
+    CUtensorMap map;
+    if (!make_act_rows_map(&map, x, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
+                           static_cast<uint64_t>(ldx)))
+        return FP8_ERR_CUDA;
+    QaParams p{};
+    p.rows = M;
+    p.nkb = K / 128;
+    p.nboxes = ((M + kQaRows - 1) / kQaRows) * p.nkb;
+    p.q = q; p.ldq = ldq;
+    p.s = sa; p.s_stride_m = sa_stride_m; p.s_stride_kb = sa_stride_kb;
+    p.dest = dest; p.topk = topk; p.out_rows = out_rows;
+    const int64_t ctas = (p.nboxes + kQaWarps - 1) / kQaWarps;
+    const unsigned grid = static_cast<unsigned>(ctas < sms ? ctas : sms);
+    if (dest)
+        quant_act_rows_kernel<true><<<grid, kQaThreads, kQaSmemBytes, stream>>>(map, p);
+    else
+        quant_act_rows_kernel<false><<<grid, kQaThreads, kQaSmemBytes, stream>>>(map, p);
+    return launch_status();
 }
 
 template <typename T, int kMode>
@@ -337,11 +438,20 @@ fp8_status_t dense_gemm(const uint8_t* a, int64_t lda, const float* sa, int64_t 
     p.nkb = static_cast<int>(K / 128);
     p.num_mt = static_cast<int>(num_mt);
     p.num_nt = static_cast<int>(num_nt);
-    // Bands of m-tiles whose A rows (band_m x 256 rows x K bytes) stay in
-    // L2 (about 40 MB of the 126 MB) while the pairs walk across N: B is
-    // then read from HBM once per band, A once.
-    const int64_t band = (int64_t{40} << 20) / (static_cast<int64_t>(kPairBM) * K);
-    p.band_m = static_cast<int>(band < 1 ? 1 : (band > num_mt ? num_mt : band));
+    // Tile raster for L2 reuse.  The smaller operand is cut into bands that
+    // stay in L2 (at most kL2BandBytes of the 126 MB) while the pairs walk
+    // across the larger one: the band operand is read from HBM once, the
+    // streamed one once per band.  Bands are balanced (equal tile counts).
+    const int64_t a_bytes = num_mt * static_cast<int64_t>(kPairBM) * K;
+    const int64_t b_bytes = num_nt * static_cast<int64_t>(kBN) * K;
+    const bool band_over_n = b_bytes < a_bytes;
+    const int64_t tiles = band_over_n ? num_nt : num_mt;
+    const int64_t panel = (band_over_n ? kBN : kPairBM) * K;     // bytes of one tile's panel
+    int64_t nbands = (tiles * panel + kL2BandBytes - 1) / kL2BandBytes;
+    nbands = nbands < 1 ? 1 : (nbands > tiles ? tiles : nbands);
+    const int band = static_cast<int>((tiles + nbands - 1) / nbands);
+    p.band_m = band_over_n ? 1 : band;
+    p.band_n = band_over_n ? band : 0;
     p.offsets = nullptr; p.G = 1;
     const int64_t pairs = grid_for(num_mt * num_nt, g_dev[dev].max_pairs, 1);
     return launch_pair_gemm<false, kQuantOut, kColScaleB>(tmA, tmB, p, pairs, c_type, stream);
@@ -386,6 +496,29 @@ fp8_status_t fp8_quantize_act_1x128_gather(const void* x, fp8_in_t x_type, int64
     return launch_status();
 }
 
+fp8_status_t fp8_quantize_act_1x128_scatter(const void* x, fp8_in_t x_type, int64_t T, int64_t K,
+                                            int64_t ldx, const int32_t* dest, int64_t topk,
+                                            uint8_t* q, int64_t R, int64_t ldq, float* sa,
+                                            int64_t sa_stride_m, int64_t sa_stride_kb,
+                                            fp8_stream_t stream) {
+    const int es = elem_size_in(x_type);
+    if (es == 0) return FP8_ERR_DTYPE;
+    if (T < 0 || R < 0 || K < 0 || K % 128 != 0 || topk < 0) return FP8_ERR_SHAPE;
+    if (T == 0 || K == 0 || topk == 0) return FP8_OK;
+    if (x_type != FP8_IN_BF16) return FP8_ERR_DTYPE;
+    if (!x || !dest || (R > 0 && (!q || !sa))) return FP8_ERR_NULL;
+    if (ldx < K || ldq < K || sa_stride_m < 0 || sa_stride_kb < 0) return FP8_ERR_LAYOUT;
+    if (!aligned16(x) || (ldx * es) % 16 != 0 || !aligned4(dest) ||
+        (R > 0 && (!aligned32(q) || ldq % 32 != 0 || !aligned4(sa))))
+        return FP8_ERR_ALIGN;
+    if (T > INT32_MAX || R > INT32_MAX || topk > INT32_MAX / (T > 0 ? T : 1)) return FP8_ERR_SHAPE;
+    int dev, sms;
+    fp8_status_t st = current_device(&dev, &sms);
+    if (st != FP8_OK) return st;
+    return launch_quant_act_rows(x, T, K, ldx, q, ldq, sa, sa_stride_m, sa_stride_kb, sms, stream,
+                                 dest, topk, R);
+}
+
 fp8_status_t fp8_dequantize(const uint8_t* q, int64_t rows, int64_t cols, int64_t ldq,
                             const float* s, int64_t s_stride_r, int64_t s_stride_c, int tile_rows,
                             void* out, fp8_out_t out_type, int64_t ldo, fp8_stream_t stream) {
@@ -407,12 +540,13 @@ fp8_status_t fp8_dequantize(const uint8_t* q, int64_t rows, int64_t cols, int64_
     if (gy > rows) gy = rows;
     if (gy > 65535) gy = 65535;
     const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
+    const int tile_shift = tile_rows == 128 ? 7 : 0;
     if (out_type == FP8_OUT_BF16)
         dequant_kernel<true><<<grid, kDqThreads, 0, stream>>>(q, rows, cols, ldq, s, s_stride_r,
-                                                              s_stride_c, tile_rows, out, ldo);
+                                                              s_stride_c, tile_shift, out, ldo);
     else
         dequant_kernel<false><<<grid, kDqThreads, 0, stream>>>(q, rows, cols, ldq, s, s_stride_r,
-                                                               s_stride_c, tile_rows, out, ldo);
+                                                               s_stride_c, tile_shift, out, ldo);
     return launch_status();
 }
 
@@ -448,6 +582,10 @@ fp8_status_t fp8_quantize_act_1x128(const void* x, fp8_in_t x_type, int64_t M, i
     int dev, sms;
     fp8_status_t st = current_device(&dev, &sms);
     if (st != FP8_OK) return st;
+    // bf16 rows whose codes can leave as 32-byte stores: one row per thread.
+    if (x_type == FP8_IN_BF16 && aligned32(q) && ldq % 32 == 0)
+        return launch_quant_act_rows(x, M, K, ldx, q, ldq, sa, sa_stride_m, sa_stride_kb, sms,
+                                     stream);
     QsParams p{};
     p.rows = M; p.cols = K;
     p.nbr = (M + 127) / 128; p.nbc = K / 128;
@@ -473,6 +611,11 @@ fp8_status_t fp8_quantize_weight_128x128(const void* w, fp8_in_t w_type, int64_t
     int dev, sms;
     fp8_status_t st = current_device(&dev, &sms);
     if (st != FP8_OK) return st;
+    // bf16 weights whose codes can leave as 32-byte stores: one block row per
+    // thread.
+    if (w_type == FP8_IN_BF16 && aligned32(q) && ldq % 32 == 0)
+        return launch_quant_weight_rows(w, K, N, ldw, q, transpose_out, ldq, sb, sb_stride_kb,
+                                        sb_stride_nb, sms, stream);
     QsParams p{};
     p.rows = K; p.cols = N;
     p.nbr = K / 128; p.nbc = N / 128;
@@ -639,6 +782,7 @@ fp8_status_t fp8_grouped_gemm(const uint8_t* a, int64_t lda, const float* sa,
     p.num_mt = 0;
     p.num_nt = static_cast<int>(num_nt);
     p.band_m = 1;
+    p.band_n = 0;
     p.offsets = offsets; p.G = G;
     if (use_pair)
         return launch_pair_gemm<true>(tmA, tmB, p, grid_for(max_mt * num_nt, g_dev[dev].max_pairs, 1),
@@ -651,6 +795,21 @@ fp8_status_t fp8_grouped_gemm(const uint8_t* a, int64_t lda, const float* sa,
         blockscaled_gemm_kernel<true, false>
             <<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, stream>>>(tmA, tmB, p);
     return launch_status();
+}
+
+fp8_status_t fp8_set_wait_limit(int64_t cycles) {
+    int dev, sms;
+    fp8_status_t st = current_device(&dev, &sms);
+    if (st != FP8_OK) return st;
+    if (cycles < 0) return FP8_ERR_SHAPE;
+    const long long v = cycles == 0 ? kWaitLimitCycles : static_cast<long long>(cycles);
+    // Synchronous copy: no kernel of this device runs with a half-written limit.
+    if (cudaDeviceSynchronize() != cudaSuccess ||
+        cudaMemcpyToSymbol(g_wait_limit_cycles, &v, sizeof v) != cudaSuccess) {
+        cudaGetLastError();
+        return FP8_ERR_CUDA;
+    }
+    return FP8_OK;
 }
 
 fp8_status_t fp8_get_device_error(fp8_stream_t stream, fp8_status_t* code) {

@@ -89,7 +89,8 @@ struct GemmParams {
     int nkb;         // K / 128
     int num_nt;      // ceil(N / kBN)
     int num_mt;      // dense only: ceil(M / kBM)
-    int band_m;      // dense raster: m-tiles per band
+    int band_m;      // dense raster: m-tiles per band (band_n == 0)
+    int band_n;      // dense raster: n-tiles per band, or 0 for bands of m-tiles
     const int32_t* offsets;  // grouped only: [G + 1]
     int G;
     // Quantized output (fp8_blockscaled_gemm_quant): codes [M, ldqc] and
@@ -137,24 +138,44 @@ struct TileCoord {
 // counter; the device-wide %globaltimer is slow to read and would delay the
 // reaction to a completed barrier).  2^31 cycles is about one second at the
 // B200's 1.9 GHz and a few seconds at its lowest clocks.
+// The limit of the waits that can abort (bounded_wait) is read from a device
+// variable, kWaitLimitCycles unless fp8_set_wait_limit() changed it: a test
+// shortens it to make real waits run out and exercise the abort path.  The
+// drains below always keep kWaitLimitCycles.
 constexpr long long kWaitLimitCycles = 1ll << 31;
 constexpr int kPollsPerClockCheck = 64;
+
+__device__ long long g_wait_limit_cycles = kWaitLimitCycles;
 
 __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity,
                                              volatile int* abort_flag) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const long long t0 = clock64();
-    while (true) {
-        for (int i = 0; i < kPollsPerClockCheck; ++i)
-            if (mbar_try_wait(a, parity)) return true;
-        if (*abort_flag) return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
+    // Constant while any kernel runs (set only with the device idle): a
+    // read-only cached load, issued here and needed only at the first
+    // clock comparison.
+    const long long limit = __ldg(&g_wait_limit_cycles);
+    for (int i = 1;; ++i) {
+        if (mbar_try_wait(a, parity)) return true;
+        // The clock every poll (a register read); the CTA's abort flag (a
+        // shared-memory load) every kPollsPerClockCheck polls.
+        if (i % kPollsPerClockCheck == 0 && *abort_flag) return false;
+        if (clock64() - t0 > limit) {
             *abort_flag = 1;
             record_device_error(kDevErrTimeout);
             return false;
         }
     }
+}
+
+// bounded_wait by every lane of a converged warp, decided for the warp as a
+// whole: true only if every lane saw the phase complete, so that all lanes
+// leave a loop on an abandoned wait together.
+__device__ __forceinline__ bool bounded_wait_warp(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort_flag) {
+    const bool ok = bounded_wait(bar, parity, abort_flag);
+    return __all_sync(0xFFFFFFFFu, ok);
 }
 
 // Same, ignoring the abort flag: used to drain copies, MMAs and arrivals
@@ -217,15 +238,28 @@ __device__ __forceinline__ TileCoord decode_tile(int t, const GemmParams& p,
                                                  const GroupTables* gt) {
     TileCoord tc;
     if (!kGrouped) {
-        // Bands of band_m m-tiles; inside a band, m runs fastest so that the
-        // CTAs of one wave share both A rows and B columns through L2.
-        const int per_band = p.band_m * p.num_nt;
-        const int band = t / per_band;
-        const int within = t - band * per_band;
-        const int bm0 = band * p.band_m;
-        const int bm = min(p.band_m, p.num_mt - bm0);
-        const int nt = within / bm;
-        const int mt = bm0 + (within - nt * bm);
+        // Bands of band_m m-tiles (the A rows of a band stay in L2 while B
+        // streams past them), m fastest inside a band; or bands of band_n
+        // n-tiles (the B rows stay, A streams), n fastest.  Either way the
+        // CTAs of one wave share both A rows and B rows through L2.
+        int mt, nt;
+        if (p.band_n == 0) {
+            const int per_band = p.band_m * p.num_nt;
+            const int band = t / per_band;
+            const int within = t - band * per_band;
+            const int bm0 = band * p.band_m;
+            const int bm = min(p.band_m, p.num_mt - bm0);
+            nt = within / bm;
+            mt = bm0 + (within - nt * bm);
+        } else {
+            const int per_band = p.band_n * p.num_mt;
+            const int band = t / per_band;
+            const int within = t - band * per_band;
+            const int bn0 = band * p.band_n;
+            const int bn = min(p.band_n, p.num_nt - bn0);
+            mt = within / bn;
+            nt = bn0 + (within - mt * bn);
+        }
         tc.m0 = static_cast<int64_t>(mt) * kTileM;
         tc.row_end = p.M;
         tc.n0 = static_cast<int64_t>(nt) * kBN;
@@ -344,7 +378,14 @@ __device__ __forceinline__ void store_row_quantized(const GemmParams& p, const f
 // The warp stages the 128 sb values of its columns for chunk kb + 1 in
 // `sb_stage` ([2][128] floats of this warp) by cp.async while it promotes
 // chunk kb.
-template <bool kOutBf16, bool kQuantOut = false, bool kColScaleB = false, typename Release>
+//
+// kHalves (CTA-pair kernel): each chunk's partial arrives as two 128-column
+// halves of its 256-column TMEM buffer, half j holding columns
+// [64 j, 64 j + 64) of each 128-column slice of the tile; half j has its
+// own "full" barrier tfull[2 buf + j] and is released (release(2 buf + j))
+// as soon as the warp has read its 64 columns of it.
+template <bool kOutBf16, bool kQuantOut = false, bool kColScaleB = false, bool kHalves = false,
+          typename Release>
 __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, uint64_t* tfull,
                                               volatile int* abort_flag, uint32_t tmem_base,
                                               uint32_t t_lane, int h, int lane, int64_t row,
@@ -402,7 +443,51 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, uint64_t* tfu
         }
 
         const uint32_t buf = chunk & 1u;
-        if (!bounded_wait(&tfull[buf], (chunk >> 1) & 1u, abort_flag)) {
+        if constexpr (kHalves) {
+            // Two halves, each read in one round trip (two loads of 32
+            // columns), released, then promoted.
+            bool ok = true;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                if (!bounded_wait_warp(&tfull[2 * buf + j], (chunk >> 1) & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t taddr = tmem_base + t_lane + buf * kBN + j * 128 + h * 64;
+                tmem_ld_32x32b_x32(taddr, pa);
+                tmem_ld_32x32b_x32(taddr + 32, pb);
+                tmem_wait_ld_dep(pa);
+                tmem_wait_ld_dep(pb);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) release(2 * buf + j);
+                if (j == 0) {
+                    if constexpr (kColScaleB) {
+                        promote32_cols<0>(acc, pa, sa2p, sbk);
+                        promote32_cols<32>(acc, pb, sa2p, sbk);
+                    } else {
+                        promote32<0>(acc, pa, scale);
+                        promote32<32>(acc, pb, scale);
+                    }
+                } else {
+                    if constexpr (kColScaleB) {
+                        promote32_cols<64>(acc, pa, sa2p, sbk);
+                        promote32_cols<96>(acc, pb, sa2p, sbk);
+                    } else {
+                        promote32<64>(acc, pa, scale);
+                        promote32<96>(acc, pb, scale);
+                    }
+                }
+            }
+            if (!ok) {
+                if constexpr (kColScaleB) cp_async_wait_all();
+                return false;
+            }
+            ++chunk;
+            continue;
+        }
+        if (!bounded_wait_warp(&tfull[buf], (chunk >> 1) & 1u, abort_flag)) {
             if constexpr (kColScaleB) cp_async_wait_all();
             return false;
         }

@@ -120,7 +120,7 @@ __device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& uses, int la
                                            volatile int* abort_flag) {
     __syncwarp();
     if (lane == 0) mbar_arrive(bar);
-    const bool ok = bounded_wait(bar, uses & 1u, abort_flag);
+    const bool ok = bounded_wait_warp(bar, uses & 1u, abort_flag);
     ++uses;
     return ok;
 }
@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(kQsThreads, 1)
         const int64_t i = box_of(k);
         const int stage = slot_of(k);
         const uint32_t phase = static_cast<uint32_t>((k / kSlots) & 1);
-        if (!bounded_wait(&tail->full[stage], phase, abort_flag)) break;
+        if (!bounded_wait_warp(&tail->full[stage], phase, abort_flag)) break;
         const uint8_t* box_smem = smem + stage * kBoxBytes;
         auto row_ptr = [&](int j) { return box_smem + row_in_box(j) * Cfg::kRowBytes; };
         // The group has finished reading the slot: refill it with the

@@ -1,0 +1,271 @@
+// quant_weight_kernels.cuh -- online 128x128 weight quantization of bf16
+// weights, one block row per thread:
+//   sb[kb, nb] = amax over the 128x128 block (kb, nb) of |w| / 448  (1 when 0)
+//   q          = E4M3_RNE_satfinite(w / sb)   written [K, N] or [N, K]
+// computed on every call, bit-exact to one IEEE fp32 division per element
+// (codingmall.com "Kan du förklara rollen för FP8 precision i
+// träningsprocessen för DeepSeek-V3", "Finkornig kvantisering",
+// "Online-kvantisering"; holysheep.ai "FP8 混精度训练 DeepSeek 671B" (zh),
+// 2.2).
+//
+// HBM-bound streaming.  One persistent CTA per SM holds kQwGroups groups of
+// 4 warps; a group walks its own sequence of 128x128 blocks through a ring of
+// kQwSlots shared-memory slots (32 KB each):
+//   * the group's first thread fills a slot with two TMA loads of 128 rows x
+//     64 bf16 (128-byte swizzle: 16-byte chunk c of row r sits at chunk
+//     c ^ (r % 8), so 8 lanes reading chunk c of 8 consecutive rows hit 8
+//     distinct bank groups);
+//   * thread t of the group takes block row t into 64 registers, reduces it
+//     with packed |max|, and the warp and then the group (through shared
+//     memory and a bounded group barrier) combine the block's amax;
+//   * every thread computes the block's scale and reciprocal and encodes its
+//     row with the FMA-corrected quotient (exact for bf16);
+//   * [K, N] output: the row's 128 codes leave as four 32-byte stores;
+//   * [N, K] output: the codes go through the slot just read (now free) as a
+//     word array U[g][k] (word g of row k = codes of columns 4g..4g+3,
+//     16-byte chunks swizzled by g), then thread n gathers byte n % 4 of
+//     words U[n / 4][k] for every k (byte permutes) and writes output row n
+//     as four 32-byte stores.  The slot is refilled one block later.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "gemm_kernels.cuh"        // bounded_wait_warp, record_device_error
+#include "quant_act_kernels.cuh"   // bf16x2_absmax, stg256_cs, lds128_addr
+#include "quant_kernels.cuh"       // Raw8, encode8_corrected, scale_from_amax
+
+namespace fp8fg {
+
+constexpr int kQwGroups = 2;                      // groups of 4 warps per CTA
+constexpr int kQwSlots = 3;
+constexpr int kQwHalfBytes = 128 * 128;           // 128 rows x 64 bf16
+constexpr int kQwBlockBytes = 2 * kQwHalfBytes;   // 32 KB: a 128x128 bf16 block
+constexpr int kQwThreads = kQwGroups * 128;
+
+struct QwSmemTail {
+    uint64_t full[kQwGroups][kQwSlots];   // slot filled (TMA bytes)
+    uint64_t gbar[kQwGroups];             // group barrier: 4 warp arrivals
+    uint32_t red[kQwGroups][2][4];        // per warp packed |max|, by block parity
+    int abort_flag;
+};
+
+constexpr size_t kQwSmemBytes =
+    1024 /* alignment slack */ + kQwGroups * kQwSlots * kQwBlockBytes + sizeof(QwSmemTail);
+
+struct QwParams {
+    int64_t nbr, nbc;          // blocks along K (rows of w) and N (columns)
+    int64_t nblocks;           // nbr * nbc
+    uint8_t* q;
+    int64_t ldq;
+    float* s;
+    int64_t s_stride_kb, s_stride_nb;
+};
+
+// Barrier of the 4 warps of a group (an mbarrier, so that the wait is
+// bounded); `uses` counts this thread's passes (the phase parity).
+__device__ __forceinline__ bool qw_group_sync(uint64_t* bar, uint32_t& uses, int lane,
+                                              volatile int* abort_flag) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar);
+    const bool ok = bounded_wait_warp(bar, uses & 1u, abort_flag);
+    ++uses;
+    return ok;
+}
+
+// Shared word address of U[g][k] in a slot: row g (512 bytes) of 128 words,
+// 16-byte chunk (k / 4) stored at chunk (k / 4) ^ (g % 8).
+__device__ __forceinline__ uint32_t qw_u_addr(uint32_t base, uint32_t g, uint32_t k) {
+    return base + g * 512u + ((((k >> 2) ^ (g & 7u)) << 4) | ((k & 3u) << 2));
+}
+
+template <bool kTransposed>
+__global__ void __launch_bounds__(kQwThreads, 1)
+    quant_weight_rows_kernel(const __grid_constant__ CUtensorMap tm_in, const QwParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    QwSmemTail* tail =
+        reinterpret_cast<QwSmemTail*>(smem + kQwGroups * kQwSlots * kQwBlockBytes);
+    volatile int* abort_flag = &tail->abort_flag;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int g = warp >> 2;              // group
+    const int wg = warp & 3;              // warp within the group
+    const int t = threadIdx.x & 127;      // thread within the group = block row
+    if (threadIdx.x == 0) {
+        for (int gi = 0; gi < kQwGroups; ++gi) {
+            for (int s = 0; s < kQwSlots; ++s) mbar_init(&tail->full[gi][s], 1);
+            mbar_init(&tail->gbar[gi], 4);
+        }
+        tail->abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_in);
+    }
+    __syncthreads();
+
+    // Group-major numbering across the grid, so that surplus blocks land on
+    // different SMs.
+    const int64_t gg = static_cast<int64_t>(g) * gridDim.x + blockIdx.x;
+    const int64_t ng = static_cast<int64_t>(kQwGroups) * gridDim.x;
+    const int64_t count = p.nblocks > gg ? (p.nblocks - 1 - gg) / ng + 1 : 0;
+    uint8_t* ring = smem + g * kQwSlots * kQwBlockBytes;
+    uint64_t* full = tail->full[g];
+    uint32_t uses = 0;
+
+    // Block b = gg + k ng is (b / nbc, b % nbc); cursors advance by ng.
+    const int64_t step_r = ng / p.nbc;
+    const int64_t step_c = ng - step_r * p.nbc;
+    auto advance = [&](int64_t& br, int64_t& bc) {
+        br += step_r;
+        bc += step_c;
+        if (bc >= p.nbc) {
+            bc -= p.nbc;
+            ++br;
+        }
+    };
+    int64_t i_br = gg / p.nbc, i_bc = gg - (gg / p.nbc) * p.nbc;   // next block to issue
+    int64_t c_br = i_br, c_bc = i_bc;                               // next block to consume
+
+    auto issue = [&](int64_t k) {   // thread 0 of the group: block k into slot k % kQwSlots
+        const int slot = static_cast<int>(k % kQwSlots);
+        uint8_t* dst = ring + slot * kQwBlockBytes;
+        mbar_arrive_expect_tx(&full[slot], kQwBlockBytes);
+        const int32_t x = static_cast<int32_t>(i_bc * 128);
+        const int32_t y = static_cast<int32_t>(i_br * 128);
+        tma_load_2d(dst, &tm_in, &full[slot], x, y);
+        tma_load_2d(dst + kQwHalfBytes, &tm_in, &full[slot], x + 64, y);
+        advance(i_br, i_bc);
+    };
+    if (t == 0)
+        for (int64_t k = 0; k < kQwSlots && k < count; ++k) issue(k);
+
+    const uint32_t swz = static_cast<uint32_t>(t & 7);
+    for (int64_t k = 0; k < count; ++k) {
+        const int slot = static_cast<int>(k % kQwSlots);
+        if (!bounded_wait_warp(&full[slot], static_cast<uint32_t>((k / kQwSlots) & 1), abort_flag))
+            break;
+        const uint32_t slot_addr = smem_u32(ring + slot * kQwBlockBytes);
+        const uint32_t row_addr = slot_addr + t * 128;
+        Raw8<uint16_t> raw[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+            raw[c].a = lds128_addr(row_addr + (c >> 3) * kQwHalfBytes +
+                                   (((static_cast<uint32_t>(c) & 7u) ^ swz) << 4));
+        uint32_t m[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+            m[c] = bf16x2_absmax(bf16x2_absmax(raw[c].a.x, raw[c].a.y),
+                                 bf16x2_absmax(raw[c].a.z, raw[c].a.w));
+#pragma unroll
+        for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+            for (int c = 0; c < w; ++c) m[c] = bf16x2_absmax(m[c], m[c + w]);
+        uint32_t wm = m[0];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            wm = bf16x2_absmax(wm, __shfl_xor_sync(0xFFFFFFFFu, wm, off));
+        const int par = static_cast<int>(k & 1);
+        if (lane == 0) tail->red[g][par][wg] = wm;
+        // After this barrier every row of the block is in registers and the
+        // four warp maxima are visible.
+        if (!qw_group_sync(&tail->gbar[g], uses, lane, abort_flag)) break;
+        uint32_t bm = bf16x2_absmax(bf16x2_absmax(tail->red[g][par][0], tail->red[g][par][1]),
+                                    bf16x2_absmax(tail->red[g][par][2], tail->red[g][par][3]));
+        bm &= 0x7FFF7FFFu;
+        const float amax = fmaxf(__uint_as_float(bm << 16), __uint_as_float(bm & 0xFFFF0000u));
+        if (t == 0) {
+            if (!kTransposed) {
+                // [K, N]: the slot just read takes the block kQwSlots ahead.
+                if (k + kQwSlots < count) issue(k + kQwSlots);
+            } else if (k > 0 && k - 1 + kQwSlots < count) {
+                // [N, K]: the previous block's slot, whose transpose buffer
+                // every thread has finished reading (it passed this barrier).
+                issue(k - 1 + kQwSlots);
+            }
+        }
+
+        const int64_t br = c_br, bc = c_bc;
+        advance(c_br, c_bc);
+        const float s = scale_from_amax(amax);
+        const float r = __frcp_rn(s);
+        uint32_t codes[32];
+        if (corrected_path_ok(s)) {
+            const uint64_t s2 = f2_pack(s, s);
+            const uint64_t neg_r2 = f2_pack(-r, -r);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                uint64_t n[4];
+                raw[c].to_neg_pairs(n);
+                const uint2 cc = encode8_corrected(n, s2, neg_r2);
+                codes[2 * c] = cc.x;
+                codes[2 * c + 1] = cc.y;
+            }
+        } else {
+            // Scale off the corrected quotient's proven range: IEEE division.
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                float v[8];
+                raw[c].to_float(v);
+                codes[2 * c] = encode2_exact(v[0], v[1], s) | (encode2_exact(v[2], v[3], s) << 16);
+                codes[2 * c + 1] =
+                    encode2_exact(v[4], v[5], s) | (encode2_exact(v[6], v[7], s) << 16);
+            }
+        }
+        if (t == 0) p.s[br * p.s_stride_kb + bc * p.s_stride_nb] = s;
+
+        if constexpr (!kTransposed) {
+            uint8_t* dst = p.q + (br * 128 + t) * p.ldq + bc * 128;
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const uint32_t w[8] = {codes[8 * q4], codes[8 * q4 + 1], codes[8 * q4 + 2],
+                                       codes[8 * q4 + 3], codes[8 * q4 + 4], codes[8 * q4 + 5],
+                                       codes[8 * q4 + 6], codes[8 * q4 + 7]};
+                stg256_cs(dst + 32 * q4, w);
+            }
+        } else {
+            // Codes word gi of row t (columns 4gi..4gi+3) -> U[gi][t].
+#pragma unroll
+            for (int gi = 0; gi < 32; ++gi)
+                asm volatile("st.shared.u32 [%0], %1;" ::"r"(qw_u_addr(slot_addr, gi, t)),
+                             "r"(codes[gi])
+                             : "memory");
+            if (!qw_group_sync(&tail->gbar[g], uses, lane, abort_flag)) break;
+            // Output row n = t: byte (n % 4) of U[n / 4][k] for k = 0..127.
+            const uint32_t gi = static_cast<uint32_t>(t) >> 2;
+            const uint32_t sel = static_cast<uint32_t>(t) & 3u;
+            // byte_perm selectors: byte `sel` of each of two words into the
+            // low two bytes, then two such halves into one word.
+            const uint32_t pick = sel | ((sel + 4u) << 4);
+            uint32_t out[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const uint4 w = lds128_addr(qw_u_addr(slot_addr, gi, 4u * j));
+                const uint32_t lo = __byte_perm(w.x, w.y, pick);
+                const uint32_t hi = __byte_perm(w.z, w.w, pick);
+                out[j] = __byte_perm(lo, hi, 0x5410);
+            }
+            // This thread's shared-memory accesses to the slot come before the
+            // TMA load that will refill it (issued after a later barrier).
+            fence_proxy_async_shared();
+            uint8_t* dst = p.q + (bc * 128 + t) * p.ldq + br * 128;
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const uint32_t w[8] = {out[8 * q4], out[8 * q4 + 1], out[8 * q4 + 2],
+                                       out[8 * q4 + 3], out[8 * q4 + 4], out[8 * q4 + 5],
+                                       out[8 * q4 + 6], out[8 * q4 + 7]};
+                stg256_cs(dst + 32 * q4, w);
+            }
+        }
+    }
+    // After an abandoned wait a fill may still be in flight: let it land
+    // before the CTA leaves (every fill is consumed on the normal path).
+    if (*abort_flag) {
+        const long long t0 = clock64();
+        while (clock64() - t0 < (1ll << 22)) {
+        }
+    }
+}
+
+}  // namespace fp8fg

@@ -118,6 +118,40 @@ FP8FG_API fp8_status_t fp8_quantize_act_1x128_gather(const void* x, fp8_in_t x_t
                                                      int64_t sa_stride_kb, fp8_stream_t stream);
 
 /*
+ * fp8_quantize_act_1x128_scatter -- the MoE dispatch in token order: each
+ * input row (token) t is quantized once, as fp8_quantize_act_1x128 would,
+ * and its codes and scales are written to every output row named by
+ * dest[t * topk + j], j < topk.  With dest the inverse of a gather's `rows`
+ * (dest[t * topk + j] = r exactly when rows[r] = t), the output equals that
+ * of fp8_quantize_act_1x128_gather bit for bit, but every token is read and
+ * quantized once instead of once per destination.
+ * [KB] "Finkornig kvantisering", "Online-kvantisering"; [HS] 2.2.
+ *
+ *  x        device bf16 [T, ldx]; 16-byte aligned, ldx * 2 % 16 == 0,
+ *           ldx >= K.  fp32 input gives FP8_ERR_DTYPE (use the gather form).
+ *  T, K     T >= 0 tokens; K >= 0 a multiple of 128.
+ *  dest     device int32 [T, topk] (row-major, 4-byte aligned): output rows
+ *           of token t; -1 marks no destination.  Any other value outside
+ *           [0, R) is skipped and records FP8_ERR_SHAPE in the device error
+ *           word.  An output row named twice receives one of the writers'
+ *           tiles (which one is undefined); rows named by no entry are not
+ *           written.
+ *  topk     >= 0 destinations per token (0: nothing to do).
+ *  q        device codes [R, ldq]; 32-byte aligned and ldq a multiple of 32
+ *           (the codes leave as 32-byte stores), ldq >= K.
+ *  R        rows of q and sa.
+ *  sa       device fp32, sa[r * sa_stride_m + kb * sa_stride_kb], 4-byte aligned.
+ *  Errors: FP8_ERR_NULL, FP8_ERR_SHAPE, FP8_ERR_ALIGN, FP8_ERR_DTYPE,
+ *          FP8_ERR_LAYOUT, FP8_ERR_DEVICE, FP8_ERR_CUDA.
+ */
+FP8FG_API fp8_status_t fp8_quantize_act_1x128_scatter(const void* x, fp8_in_t x_type, int64_t T,
+                                                      int64_t K, int64_t ldx,
+                                                      const int32_t* dest, int64_t topk,
+                                                      uint8_t* q, int64_t R, int64_t ldq,
+                                                      float* sa, int64_t sa_stride_m,
+                                                      int64_t sa_stride_kb, fp8_stream_t stream);
+
+/*
  * fp8_quantize_weight_128x128 -- online fine-grained weight quantization.
  * [KB] "Finkornig kvantisering" (weights in 128x128 blocks, each scaled on
  * its own), "Online-kvantisering"; [HS] 2.2.
@@ -320,11 +354,36 @@ FP8FG_API const char* fp8_status_string(fp8_status_t status);
  * fp8_get_device_error -- synchronizes `stream`, then reads and clears the
  * current device's error word.  Kernels record into it when a bounded wait
  * gives up (FP8_ERR_DEVICE_TIMEOUT; the kernel then stops early and its
- * outputs are undefined) or when the grouped GEMM meets invalid offsets
- * (FP8_ERR_SHAPE).  *code receives the recorded status (FP8_OK if none).
- * Returns FP8_ERR_CUDA if the synchronization or the read fails.
+ * outputs are undefined) or when the grouped GEMM or the gathering
+ * quantizer meets invalid offsets or row indices (FP8_ERR_SHAPE).  *code
+ * receives the recorded status (FP8_OK if none).
+ *
+ * There is ONE error word per device, shared by every stream and every call
+ * of this library on that device: the first error recorded since the last
+ * read is kept (later ones are dropped), and whoever reads it clears it.
+ * Only `stream` is synchronized, so a kernel still running on another
+ * stream may record an error after this read.  Callers that use several
+ * streams should read the word only after synchronizing all of them, and
+ * from one place.
+ * Returns FP8_ERR_NULL if `code` is NULL, FP8_ERR_CUDA if the
+ * synchronization or the read fails.
  */
 FP8FG_API fp8_status_t fp8_get_device_error(fp8_stream_t stream, fp8_status_t* code);
+
+/*
+ * fp8_set_wait_limit -- sets, for the current device, how many SM clock
+ * cycles any wait of this library's kernels may last before the kernel
+ * gives up (records FP8_ERR_DEVICE_TIMEOUT, waits for its own copies and
+ * tensor-core work in flight, releases its tensor memory and returns, so
+ * that the context stays usable).  cycles == 0 restores the default,
+ * 2^31 cycles (about one second at the B200's clock).  A test sets a few
+ * hundred cycles to make real waits run out and exercise that path; the
+ * results of calls made under such a limit are undefined.
+ * Synchronizes the device before the change.  Not for use while other
+ * threads queue work on the device.
+ * Errors: FP8_ERR_SHAPE (cycles < 0), FP8_ERR_DEVICE, FP8_ERR_CUDA.
+ */
+FP8FG_API fp8_status_t fp8_set_wait_limit(int64_t cycles);
 
 #ifdef __cplusplus
 }

@@ -243,8 +243,12 @@ def gemm_ref_colscale(qa, sa, qb, sb_cols):
     """Block-scaled GEMM whose B scales are per output column and chunk (the
     weight-gradient product dW = X^T dY, both operands quantized in 1x128
     tiles along the contraction): C[i, n] = sum_k (sa[i, k/128] dec(qa[i, k]))
-    (sb_cols[n, k/128] dec(qb[n, k])), in fp64 (products of E4M3 values and
-    fp32 scales are exact there), and T = sum_k |.| of the same products
+    (sb_cols[n, k/128] dec(qb[n, k])), in fp64, and T = sum_k |.| of the
+    same products.  Each dequantized operand (a 4-bit E4M3 significand times
+    a 24-bit fp32 scale) is exact in fp64, but the product of two such
+    operands can carry up to 56 significant bits, so it and the sum are
+    rounded to fp64: a relative error near 2^-53 per term, far inside the
+    1e-3 T acceptance bound
     ([KB] "Ökad ackumuleringsprecision"; [HS] 2.2 dequantize).  qa [I, K],
     qb [N, K] (K-major), sa [I, K/128], sb_cols [N, K/128].
     Returns (C, T) as fp64 [I, N]."""

@@ -84,6 +84,16 @@ def moe_routing(tokens, experts, topk, seed, device="cpu"):
     return token_of[order].contiguous(), offsets.to(torch.int32)
 
 
+def moe_dispatch_dest(token_of_row, tokens, topk):
+    """The routing of ``moe_routing`` in token order: dest int32 [tokens,
+    topk] with dest[t, j] the j-th expert-sorted row (in row order) that
+    holds token t, the inverse of ``token_of_row``.  Index bookkeeping only."""
+    R = token_of_row.numel()
+    rows = torch.arange(R, device=token_of_row.device)
+    perm = torch.argsort(token_of_row.long() * R + rows)      # by token, then row
+    return perm.to(torch.int32).view(tokens, topk).contiguous()
+
+
 @dataclass
 class Workload:
     name: str

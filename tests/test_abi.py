@@ -149,6 +149,7 @@ def test_valid_arguments_without_gpu_report_device_error(L):
     assert gemm(L) == 6
     code = ctypes.c_int(0)
     assert L.fp8_get_device_error(None, ctypes.byref(code)) == 6
+    assert L.fp8_set_wait_limit(0) == 6
 
 
 def test_dequantize_argument_errors(L):
@@ -206,6 +207,34 @@ def test_gather_quant_argument_errors(L):
     assert call(ldq=64) == 4
     assert call(ldx=132) == 3          # ldx * 2 bytes % 16
     assert call(rows=vp(base + 2)) == 3
+
+
+def test_scatter_quant_argument_errors(L):
+    vp = ctypes.c_void_p
+    buf = ctypes.create_string_buffer(4096 + 32)
+    base = (ctypes.addressof(buf) + 31) // 32 * 32
+    p = vp(base)
+
+    # x, x_type, T, K, ldx, dest, topk, q, R, ldq, sa, sa_m, sa_kb, stream
+    def call(x=p, xt=0, T=4, K=128, ldx=128, dest=p, topk=2, q=p, R=8, ldq=128, sa=p, sm=1):
+        return L.fp8_quantize_act_1x128_scatter(x, xt, T, K, ldx, dest, topk, q, R, ldq, sa, sm,
+                                                1, None)
+    assert call(xt=7) == 5
+    assert call(xt=1) == 5                  # bf16 input only
+    assert call(K=100) == 2
+    assert call(T=-1) == 2
+    assert call(topk=-1) == 2
+    assert call(T=0, x=None, dest=None) == 0   # empty: no-op
+    assert call(topk=0, dest=None) == 0
+    assert call(dest=None) == 1
+    assert call(q=None) == 1
+    assert call(ldq=64) == 4
+    assert call(ldx=64) == 4
+    assert call(sm=-1) == 4
+    assert call(q=vp(base + 16)) == 3       # codes leave as 32-byte stores
+    assert call(ldq=144) == 3               # ldq % 32
+    assert call(dest=vp(base + 2)) == 3
+    assert call(x=vp(base + 8)) == 3
 
 
 def test_act_128x1_argument_errors(L):

@@ -1,5 +1,7 @@
-"""Fused row gather + 1x128 quantization (MoE dispatch): bit-identical to the
-oracle's quantization of the gathered rows x[rows]."""
+"""Fused MoE dispatch + 1x128 quantization, in row order (gather: output row
+r from token rows[r]) and in token order (scatter: token t to output rows
+dest[t, :]): bit-identical to the oracle's quantization of the gathered
+rows x[rows]."""
 import numpy as np
 import pytest
 import torch
@@ -33,7 +35,7 @@ def test_gather_quant_equals_gather_then_quantize(cuda_lib):
 
 
 def test_invalid_index_reported_and_row_untouched(cuda_lib):
-    x = torch.randn(10, 256).bfloat16().cuda()
+    x = torch.randn(10, 256, generator=torch.Generator().manual_seed(10)).bfloat16().cuda()
     rows = torch.tensor([0, 3, 10, 9, -1], dtype=torch.int32).cuda()
     q = torch.full((5, 256), 0xAB, dtype=torch.uint8, device="cuda")
     sa = torch.full((5, 2), -3.0, device="cuda")
@@ -62,3 +64,48 @@ def test_moe_dispatch_full_size_sampled(cuda_lib, orc):
     qo, sao = orc.quantize_act_1x128(to_oracle(x[rows[pick].long()]))
     assert_codes_equal(np_u8(q[torch.from_numpy(pick).cuda()]), qo)
     assert_scales_equal(sa[torch.from_numpy(pick).cuda()].cpu().numpy(), sao)
+
+
+def _routing(T, E, topk, seed):
+    token_of, _ = synth.moe_routing(T, E, topk, seed)
+    return token_of, synth.moe_dispatch_dest(token_of, T, topk)
+
+
+@pytest.mark.parametrize("T,E,topk,K", [(1, 4, 1, 128), (33, 8, 3, 384), (300, 16, 4, 1024),
+                                        (97, 64, 11, 256), (1024, 32, 8, 7168)])
+def test_scatter_quant_matches_oracle_and_gather(cuda_lib, orc, T, E, topk, K):
+    """Token-order dispatch: every routed row equals the oracle's quantization
+    of its token, and the whole output equals the gather form's."""
+    x = synth.act_input(T, K, 1.0, 1e-2, 100.0, 7, "cpu", torch.bfloat16, tensor_id=T % 5)
+    token_of, dest = _routing(T, E, topk, 1000 + T)
+    R = T * topk
+    q, sa = cuda_lib.fp8_quantize_act_1x128_scatter(x.cuda(), dest.cuda(), R)
+    qo, sao = orc.quantize_act_1x128(to_oracle(x[token_of]))
+    assert_codes_equal(np_u8(q), qo)
+    assert_scales_equal(sa.cpu().numpy(), sao)
+    qg, sg = cuda_lib.fp8_quantize_act_1x128_gather(x.cuda(), token_of.to(torch.int32).cuda())
+    assert torch.equal(q, qg)
+    assert torch.equal(sa.view(torch.int32), sg.view(torch.int32))
+
+
+def test_scatter_skips_minus_one_and_reports_bad_rows(cuda_lib, orc):
+    """-1 entries write nothing; entries outside [0, R) record FP8_ERR_SHAPE
+    and write nothing; the valid entries are exact."""
+    T, K, R = 40, 256, 64
+    x = synth.act_input(T, K, 1.0, 1e-2, 100.0, 7, "cpu", torch.bfloat16, tensor_id=3)
+    dest = torch.full((T, 2), -1, dtype=torch.int32)
+    dest[:, 0] = torch.arange(T, dtype=torch.int32)            # token t -> row t
+    dest[5, 1] = 50
+    dest[7, 1] = R                                              # out of range
+    dest[9, 1] = -7                                             # out of range
+    q = torch.full((R, K), 0xEE, dtype=torch.uint8, device="cuda")
+    sa = torch.full((R, K // 128), -5.0, device="cuda")
+    assert cuda_lib.fp8_get_device_error() == 0
+    cuda_lib.fp8_quantize_act_1x128_scatter(x.cuda(), dest.cuda(), R, q=q, sa=sa)
+    assert cuda_lib.fp8_get_device_error() == 2
+    qo, sao = orc.quantize_act_1x128(to_oracle(x))
+    assert_codes_equal(np_u8(q[:T]), qo)
+    assert_scales_equal(sa[:T].cpu().numpy(), sao)
+    assert_codes_equal(np_u8(q[50:51]), qo[5:6])
+    untouched = [r for r in range(T, R) if r != 50]
+    assert torch.all(q[untouched] == 0xEE) and torch.all(sa[untouched] == -5.0)

@@ -41,8 +41,26 @@ def test_act_quant_strided_layouts(cuda_lib, orc):
     assert np.all(untouched[:, :64] == 0xAB) and np.all(untouched[:, 64 + K:] == 0xAB)
 
 
+@pytest.mark.parametrize("M,K", [(1, 128), (31, 256), (33, 384), (1000, 1024)])
+def test_act_quant_row_and_stream_paths_agree(cuda_lib, orc, M, K):
+    """bf16 codes written with 32-byte alignment take the one-row-per-thread
+    kernel; codes at a 16-byte offset (ldq a multiple of 16 only) take the
+    streamed 128x128-box kernel.  Both equal the oracle bit for bit."""
+    x = act(M, K, torch.bfloat16, 5 * M + K).cuda()
+    qo, sao = orc.quantize_act_1x128(to_oracle(x))
+    for offset, ld in ((0, K), (16, K + 16)):
+        qbuf = torch.full((M, ld + offset), 0xCD, dtype=torch.uint8, device="cuda")
+        q = qbuf[:, offset:offset + K]
+        _, sa = cuda_lib.fp8_quantize_act_1x128(x, q=q)
+        assert_codes_equal(np_u8(q), qo)
+        assert_scales_equal(sa.cpu().numpy(), sao)
+        rest = np_u8(qbuf)
+        assert np.all(rest[:, :offset] == 0xCD) and np.all(rest[:, offset + K:] == 0xCD)
+
+
 def test_act_quant_special_values(cuda_lib, orc):
-    x = torch.randn(8, 512) * 3
+    g = torch.Generator().manual_seed(123)
+    x = torch.randn(8, 512, generator=g) * 3
     x[0, :128] = 0.0                               # zero tile -> scale 1
     x[0, 128:256] = -0.0
     x[1, :128] = 1e-42                             # subnormal fp32 amax: amax/448 underflows
@@ -116,16 +134,20 @@ def test_quotients_at_rounding_midpoints(cuda_lib, orc, dtype):
 
 
 def test_act_quant_nan_element_smoke(cuda_lib, orc):
-    """Out of contract: a NaN element is skipped by amax and encodes to NaN."""
-    x = torch.randn(2, 256)
+    """Out of contract: a NaN element is skipped by amax and encodes to NaN
+    (fp32 and bf16 inputs, both activation kernels)."""
+    gen = torch.Generator().manual_seed(321)
+    x = torch.randn(2, 256, generator=gen)
     x[1, 17] = float("nan")
-    q, sa = cuda_lib.fp8_quantize_act_1x128(x.cuda())
-    qo, sao = orc.quantize_act_1x128(x.numpy())
-    g = np_u8(q)
-    assert (g[1, 17] & 0x7F) == 0x7F
-    g[1, 17] = qo[1, 17]
-    assert_codes_equal(g, qo)
-    assert_scales_equal(sa.cpu().numpy(), sao)
+    for dtype in (torch.float32, torch.bfloat16):
+        xd = x.to(dtype)
+        q, sa = cuda_lib.fp8_quantize_act_1x128(xd.cuda())
+        qo, sao = orc.quantize_act_1x128(to_oracle(xd))
+        g = np_u8(q)
+        assert (g[1, 17] & 0x7F) == 0x7F
+        g[1, 17] = qo[1, 17]
+        assert_codes_equal(g, qo)
+        assert_scales_equal(sa.cpu().numpy(), sao)
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
@@ -138,6 +160,26 @@ def test_weight_quant_bit_exact(cuda_lib, orc, K, N, dtype, transpose):
     qo, sbo = orc.quantize_weight_128x128(to_oracle(w), transpose_out=transpose)
     assert_codes_equal(np_u8(q), qo)
     assert_scales_equal(sb.cpu().numpy(), sbo)
+
+
+@pytest.mark.parametrize("transpose", [False, True])
+@pytest.mark.parametrize("K,N", [(128, 128), (384, 640), (1024, 256)])
+def test_weight_quant_row_and_stream_paths_agree(cuda_lib, orc, K, N, transpose):
+    """bf16 codes written with 32-byte alignment take the one-block-row-per-
+    thread kernel; codes at a 16-byte offset take the streamed box kernel.
+    Both equal the oracle bit for bit and write nothing outside q."""
+    w = synth.normal((K, N), 0.02, 2000 + K + N, "cpu", torch.bfloat16)
+    synth.scale_outliers(w, 1e-3, 100.0, 78)
+    qo, sbo = orc.quantize_weight_128x128(to_oracle(w), transpose_out=transpose)
+    rows, cols = (N, K) if transpose else (K, N)
+    for offset, ld in ((0, cols), (16, cols + 16)):
+        qbuf = torch.full((rows, ld + offset), 0xCD, dtype=torch.uint8, device="cuda")
+        q = qbuf[:, offset:offset + cols]
+        _, sb = cuda_lib.fp8_quantize_weight_128x128(w.cuda(), transpose_out=transpose, q=q)
+        assert_codes_equal(np_u8(q), qo)
+        assert_scales_equal(sb.cpu().numpy(), sbo)
+        rest = np_u8(qbuf)
+        assert np.all(rest[:, :offset] == 0xCD) and np.all(rest[:, offset + cols:] == 0xCD)
 
 
 def test_weight_quant_zero_and_strided(cuda_lib, orc):

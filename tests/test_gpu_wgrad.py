@@ -63,7 +63,7 @@ def test_act_128x1_special_values(cuda_lib, orc):
     """Zero and -0 columns (scale 1), subnormal amax (scale off the fast
     quotient's range: IEEE division), huge amax, a column at 448, NaN
     elements (out of contract: skipped by amax, NaN codes)."""
-    x = torch.randn(256, 512) * 3
+    x = torch.randn(256, 512, generator=torch.Generator().manual_seed(66)) * 3
     x[:128, 0] = 0.0
     x[:128, 1] = -0.0
     x[128:, 2] = 1e-39
