@@ -713,11 +713,16 @@ class MoE(Workload):
     unit = "TFLOP/s"
     dominant = "grouped_gemm_gate_up"
 
-    def __init__(self, fp8, device, tokens=8192, experts=256, topk=8, hidden=7168, inter=2048):
+    def __init__(self, fp8, device, tokens=8192, experts=256, topk=8, hidden=7168, inter=2048,
+                 dispatch="gather"):
         self.fp8 = fp8
         self.T, self.E, self.k, self.H, self.I = tokens, experts, topk, hidden, inter
         self.R = tokens * topk
-        self.kernels = ["quant_act_1x128_scatter_x", "grouped_gemm_gate_up", "quant_act_1x128_h",
+        # the dispatch in row order (gather: output row r <- token rows[r]) or
+        # in token order (scatter: token t -> rows dest[t, :])
+        self.dispatch = dispatch
+        self.dispatch_kernel = "quant_act_1x128_%s_x" % dispatch
+        self.kernels = [self.dispatch_kernel, "grouped_gemm_gate_up", "quant_act_1x128_h",
                         "grouped_gemm_down"]
         if device is None:
             return
@@ -753,15 +758,17 @@ class MoE(Workload):
                 "routed_rows": self.R, "gate_up": "K=%d N=%d" % (self.H, 2 * self.I),
                 "down": "K=%d N=%d" % (self.I, self.H), "out": "bf16",
                 "weights": "quantized once before timing (11.27 GB E4M3)",
-                "dispatch": "each token row quantized once inside the activation quantizer and "
-                            "written to its 8 expert-sorted rows",
+                "dispatch": ("routed rows gathered from the token rows inside the activation "
+                             "quantizer" if self.dispatch == "gather" else
+                             "each token row quantized once inside the activation quantizer and "
+                             "written to its 8 expert-sorted rows"),
                 "l2": "expert weights 11.27 GB >> L2"}
 
     def algorithmic(self):
         R, H, I, E = self.R, self.H, self.I, self.E
         return {
             # tokens read once, routed rows written (codes + scales)
-            "quant_act_1x128_scatter_x": ("bytes", self.T * H * 2 + R * H + R * (H // 128) * 4),
+            self.dispatch_kernel: ("bytes", self.T * H * 2 + R * H + R * (H // 128) * 4),
             "grouped_gemm_gate_up": ("flops", 2.0 * R * 2 * I * H),
             "quant_act_1x128_h": ("bytes", R * I * 3 + R * (I // 128) * 4),
             "grouped_gemm_down": ("flops", 2.0 * R * H * I),
@@ -781,7 +788,10 @@ class MoE(Workload):
     def step(self, marks):
         f = self.fp8
         marks(0)
-        f.fp8_quantize_act_1x128_scatter(self.x, self.dest, self.R, q=self.qx, sa=self.sx)
+        if self.dispatch == "gather":
+            f.fp8_quantize_act_1x128_gather(self.x, self.rows, q=self.qx, sa=self.sx)
+        else:
+            f.fp8_quantize_act_1x128_scatter(self.x, self.dest, self.R, q=self.qx, sa=self.sx)
         marks(1)
         f.fp8_grouped_gemm(self.qx, self.sx, self.qgu, self.sgu, self.off, c=self.cgu)
         marks(2)
@@ -792,21 +802,26 @@ class MoE(Workload):
 
     def e2e_setup(self):
         self.hx = self.x.cpu().pin_memory()
+        self.hrows = self.rows.cpu().pin_memory()
         self.hdest = self.dest.cpu().pin_memory()
         self.hh = self.h.cpu().pin_memory()
         self.hoff = self.off.cpu().pin_memory()
         self.hgu = torch.empty_like(self.cgu, device="cpu").pin_memory()
         self.hdn = torch.empty_like(self.cdn, device="cpu").pin_memory()
-        return ((self.hx.numel() + self.hh.numel()) * 2 + (self.hoff.numel() + self.hdest.numel()) * 4,
+        route = self.hrows if self.dispatch == "gather" else self.hdest
+        return ((self.hx.numel() + self.hh.numel()) * 2 + (self.hoff.numel() + route.numel()) * 4,
                 (self.hgu.numel() + self.hdn.numel()) * 2)
 
     def e2e_step(self):
         f = self.fp8
         x = self.hx.to("cuda", non_blocking=True)
-        dest = self.hdest.to("cuda", non_blocking=True)
         h = self.hh.to("cuda", non_blocking=True)
         off = self.hoff.to("cuda", non_blocking=True)
-        qx, sx = f.fp8_quantize_act_1x128_scatter(x, dest, self.R)
+        if self.dispatch == "gather":
+            qx, sx = f.fp8_quantize_act_1x128_gather(x, self.hrows.to("cuda", non_blocking=True))
+        else:
+            qx, sx = f.fp8_quantize_act_1x128_scatter(x, self.hdest.to("cuda", non_blocking=True),
+                                                      self.R)
         cgu = f.fp8_grouped_gemm(qx, sx, self.qgu, self.sgu, off)
         qh, sh = f.fp8_quantize_act_1x128(h)
         cdn = f.fp8_grouped_gemm(qh, sh, self.qdn, self.sdn, off)
@@ -872,8 +887,9 @@ def make_workload(args, fp8, device):
     """The workload object; --moe-experts E shrinks the MoE workload to E
     experts and 32 E tokens (same rows per expert), for profiler captures
     that must stay small."""
-    if args.workload == "moe" and args.moe_experts != 256:
-        return MoE(fp8, device, tokens=32 * args.moe_experts, experts=args.moe_experts)
+    if args.workload == "moe":
+        return MoE(fp8, device, tokens=32 * args.moe_experts, experts=args.moe_experts,
+                   dispatch=args.moe_dispatch)
     return WORKLOADS[args.workload](fp8, device)
 
 
@@ -1044,6 +1060,8 @@ def main():
                     help="comma list of workloads timed after the headline and reported under "
                          "'workloads' (default: all others when the headline is ffn; 'none')")
     ap.add_argument("--no-quant-error", action="store_true")
+    ap.add_argument("--moe-dispatch", choices=["gather", "scatter"], default="gather",
+                    help="MoE workload only: dispatch in row order (gather) or token order")
     ap.add_argument("--moe-experts", type=int, default=256,
                     help="MoE workload only: number of experts (tokens = 32 x experts)")
     args = ap.parse_args()

@@ -9,6 +9,7 @@
 
 #include <atomic>
 #include <cstdint>
+#include <cstring>
 #include <mutex>
 
 #include "../../include/fp8fg.h"
@@ -89,13 +90,14 @@ fp8_status_t current_device(int* dev_out, int* sms_out) {
                     }
                 }
                 const void* qa_kernels[] = {
-                    reinterpret_cast<const void*>(&quant_act_rows_kernel<false>),
-                    reinterpret_cast<const void*>(&quant_act_rows_kernel<true>),
+                    reinterpret_cast<const void*>(&quant_act_rows_kernel<kRowsPlain>),
+                    reinterpret_cast<const void*>(&quant_act_rows_kernel<kRowsScatter>),
+                    reinterpret_cast<const void*>(&quant_act_rows_kernel<kRowsGather>),
                     reinterpret_cast<const void*>(&quant_weight_rows_kernel<false>),
                     reinterpret_cast<const void*>(&quant_weight_rows_kernel<true>)};
-                const size_t qa_bytes[] = {kQaSmemBytes, kQaSmemBytes, kQwSmemBytes,
-                                           kQwSmemBytes};
-                for (int i = 0; i < 4; ++i) {
+                const size_t qa_bytes[] = {kQaSmemBytes, kQaSmemBytes, kQaSmemBytes,
+                                           kQwSmemBytes, kQwSmemBytes};
+                for (int i = 0; i < 5; ++i) {
                     if (cudaFuncSetAttribute(qa_kernels[i],
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(qa_bytes[i])) != cudaSuccess) {
@@ -335,9 +337,33 @@ fp8_status_t launch_quant_act_rows(const void* x, int64_t M, int64_t K, int64_t 
     const int64_t ctas = (p.nboxes + kQaWarps - 1) / kQaWarps;
     const unsigned grid = static_cast<unsigned>(ctas < sms ? ctas : sms);
     if (dest)
-        quant_act_rows_kernel<true><<<grid, kQaThreads, kQaSmemBytes, stream>>>(map, p);
+        quant_act_rows_kernel<kRowsScatter><<<grid, kQaThreads, kQaSmemBytes, stream>>>(map, p);
     else
-        quant_act_rows_kernel<false><<<grid, kQaThreads, kQaSmemBytes, stream>>>(map, p);
+        quant_act_rows_kernel<kRowsPlain><<<grid, kQaThreads, kQaSmemBytes, stream>>>(map, p);
+    return launch_status();
+}
+
+// Gather form: output row r <- bf16 input row rows[r] of x [src_rows, ldx],
+// fetched row by row with bulk copies (no tensor map).
+fp8_status_t launch_quant_act_rows_gather(const void* x, int64_t src_rows, int64_t K, int64_t ldx,
+                                          const int32_t* rows, int64_t R, uint8_t* q,
+                                          int64_t ldq, float* sa, int64_t sa_stride_m,
+                                          int64_t sa_stride_kb, int sms, cudaStream_t stream) {
+    CUtensorMap unused;
+    memset(&unused, 0, sizeof unused);
+    QaParams p{};
+    p.rows = R;
+    p.nkb = K / 128;
+    p.nboxes = ((R + kQaRows - 1) / kQaRows) * p.nkb;
+    p.q = q; p.ldq = ldq;
+    p.s = sa; p.s_stride_m = sa_stride_m; p.s_stride_kb = sa_stride_kb;
+    p.gidx = rows;
+    p.x = static_cast<const uint16_t*>(x);
+    p.ldx = ldx;
+    p.src_rows = src_rows;
+    const int64_t ctas = (p.nboxes + kQaWarps - 1) / kQaWarps;
+    const unsigned grid = static_cast<unsigned>(ctas < sms ? ctas : sms);
+    quant_act_rows_kernel<kRowsGather><<<grid, kQaThreads, kQaSmemBytes, stream>>>(unused, p);
     return launch_status();
 }
 
@@ -432,6 +458,8 @@ fp8_status_t dense_gemm(const uint8_t* a, int64_t lda, const float* sa, int64_t 
         return FP8_ERR_CUDA;
 
     GemmParams p = out;
+    p.c_v8 = (p.c != nullptr && aligned32(p.c) &&
+              (p.ldc * elem_size_out(c_type)) % 32 == 0) ? 1 : 0;
     p.sa = sa; p.sa_sm = sa_stride_m; p.sa_skb = sa_stride_kb;
     p.sb = sb; p.sb_sg = 0; p.sb_skb = sb_stride_kb; p.sb_snb = sb_stride_nb;
     p.M = M; p.N = N;
@@ -481,6 +509,12 @@ fp8_status_t fp8_quantize_act_1x128_gather(const void* x, fp8_in_t x_type, int64
     int dev, sms;
     fp8_status_t st = current_device(&dev, &sms);
     if (st != FP8_OK) return st;
+    // bf16 rows whose codes can leave as 32-byte stores: one row per thread,
+    // rows fetched by bulk copies.
+    if (x_type == FP8_IN_BF16 && aligned32(q) && ldq % 32 == 0 && src_rows <= INT32_MAX &&
+        R <= INT32_MAX)
+        return launch_quant_act_rows_gather(x, src_rows, K, ldx, rows, R, q, ldq, sa, sa_stride_m,
+                                            sa_stride_kb, sms, stream);
     // one half-warp per output row at a time
     const int64_t grid = grid_for((R + 15) / 16, sms, kGqMinBlocks);
     const unsigned g = static_cast<unsigned>(grid);
@@ -778,6 +812,7 @@ fp8_status_t fp8_grouped_gemm(const uint8_t* a, int64_t lda, const float* sa,
     p.sa = sa; p.sa_sm = sa_stride_m; p.sa_skb = sa_stride_kb;
     p.sb = sb; p.sb_sg = sb_stride_g; p.sb_skb = sb_stride_kb; p.sb_snb = sb_stride_nb;
     p.c = c; p.ldc = ldc; p.M = total_M; p.N = N;
+    p.c_v8 = (aligned32(c) && (ldc * elem_size_out(c_type)) % 32 == 0) ? 1 : 0;
     p.nkb = static_cast<int>(K / 128);
     p.num_mt = 0;
     p.num_nt = static_cast<int>(num_nt);

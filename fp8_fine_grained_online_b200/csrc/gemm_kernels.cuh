@@ -99,7 +99,15 @@ struct GemmParams {
     int64_t ldqc;
     float* sc;
     int64_t sc_sm, sc_snb;
+    int c_v8;        // C rows may be written as 32-byte stores (c and ldc 32-byte aligned)
 };
+
+// One 32-byte store of 8 words (the address 32-byte aligned).
+__device__ __forceinline__ void stg256(void* p, const uint32_t* w) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]),
+                 "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+}
 
 // Grouped GEMM: the persistent tile schedule, built in shared memory from
 // the device-side offsets at kernel start.
@@ -144,6 +152,7 @@ struct TileCoord {
 // drains below always keep kWaitLimitCycles.
 constexpr long long kWaitLimitCycles = 1ll << 31;
 constexpr int kPollsPerClockCheck = 64;
+constexpr int kFastPolls = 16;
 
 __device__ long long g_wait_limit_cycles = kWaitLimitCycles;
 
@@ -152,14 +161,17 @@ __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity,
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const long long t0 = clock64();
-    // Constant while any kernel runs (set only with the device idle): a
-    // read-only cached load, issued here and needed only at the first
-    // clock comparison.
+    // Fast path: most waits end within a few polls, and nothing here may
+    // wait on a memory load (the reaction to a completed phase is on the
+    // critical path of the GEMM pipeline).
+#pragma unroll 1
+    for (int i = 0; i < kFastPolls; ++i)
+        if (mbar_try_wait(a, parity)) return true;
+    // Slow path: the limit (constant while any kernel runs), the clock every
+    // poll, the CTA's abort flag every kPollsPerClockCheck polls.
     const long long limit = __ldg(&g_wait_limit_cycles);
     for (int i = 1;; ++i) {
         if (mbar_try_wait(a, parity)) return true;
-        // The clock every poll (a register read); the CTA's abort flag (a
-        // shared-memory load) every kPollsPerClockCheck polls.
         if (i % kPollsPerClockCheck == 0 && *abort_flag) return false;
         if (clock64() - t0 > limit) {
             *abort_flag = 1;
@@ -378,14 +390,7 @@ __device__ __forceinline__ void store_row_quantized(const GemmParams& p, const f
 // The warp stages the 128 sb values of its columns for chunk kb + 1 in
 // `sb_stage` ([2][128] floats of this warp) by cp.async while it promotes
 // chunk kb.
-//
-// kHalves (CTA-pair kernel): each chunk's partial arrives as two 128-column
-// halves of its 256-column TMEM buffer, half j holding columns
-// [64 j, 64 j + 64) of each 128-column slice of the tile; half j has its
-// own "full" barrier tfull[2 buf + j] and is released (release(2 buf + j))
-// as soon as the warp has read its 64 columns of it.
-template <bool kOutBf16, bool kQuantOut = false, bool kColScaleB = false, bool kHalves = false,
-          typename Release>
+template <bool kOutBf16, bool kQuantOut = false, bool kColScaleB = false, typename Release>
 __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, uint64_t* tfull,
                                               volatile int* abort_flag, uint32_t tmem_base,
                                               uint32_t t_lane, int h, int lane, int64_t row,
@@ -443,50 +448,6 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, uint64_t* tfu
         }
 
         const uint32_t buf = chunk & 1u;
-        if constexpr (kHalves) {
-            // Two halves, each read in one round trip (two loads of 32
-            // columns), released, then promoted.
-            bool ok = true;
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                if (!bounded_wait_warp(&tfull[2 * buf + j], (chunk >> 1) & 1u, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t taddr = tmem_base + t_lane + buf * kBN + j * 128 + h * 64;
-                tmem_ld_32x32b_x32(taddr, pa);
-                tmem_ld_32x32b_x32(taddr + 32, pb);
-                tmem_wait_ld_dep(pa);
-                tmem_wait_ld_dep(pb);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) release(2 * buf + j);
-                if (j == 0) {
-                    if constexpr (kColScaleB) {
-                        promote32_cols<0>(acc, pa, sa2p, sbk);
-                        promote32_cols<32>(acc, pb, sa2p, sbk);
-                    } else {
-                        promote32<0>(acc, pa, scale);
-                        promote32<32>(acc, pb, scale);
-                    }
-                } else {
-                    if constexpr (kColScaleB) {
-                        promote32_cols<64>(acc, pa, sa2p, sbk);
-                        promote32_cols<96>(acc, pb, sa2p, sbk);
-                    } else {
-                        promote32<64>(acc, pa, scale);
-                        promote32<96>(acc, pb, scale);
-                    }
-                }
-            }
-            if (!ok) {
-                if constexpr (kColScaleB) cp_async_wait_all();
-                return false;
-            }
-            ++chunk;
-            continue;
-        }
         if (!bounded_wait_warp(&tfull[buf], (chunk >> 1) & 1u, abort_flag)) {
             if constexpr (kColScaleB) cp_async_wait_all();
             return false;
@@ -524,23 +485,37 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, uint64_t* tfu
             store_row_quantized(p, acc, row, col0);
         } else if (kOutBf16) {
             __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.c) + row * p.ldc + col0;
+            uint32_t w[64];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                uint32_t w[4];
+            for (int e = 0; e < 64; ++e) {
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
+                w[e] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            if (p.c_v8) {   // whole 32-byte sectors per lane
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const __nv_bfloat162 b2 =
-                        __floats2bfloat162_rn(acc[j * 8 + 2 * e], acc[j * 8 + 2 * e + 1]);
-                    w[e] = *reinterpret_cast<const uint32_t*>(&b2);
-                }
-                reinterpret_cast<uint4*>(out)[j] = make_uint4(w[0], w[1], w[2], w[3]);
+                for (int j = 0; j < 8; ++j) stg256(out + 16 * j, w + 8 * j);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    reinterpret_cast<uint4*>(out)[j] =
+                        make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
             }
         } else {
             float* out = reinterpret_cast<float*>(p.c) + row * p.ldc + col0;
+            if (p.c_v8) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-                reinterpret_cast<float4*>(out)[j] =
-                    make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
+                for (int j = 0; j < 16; ++j) {
+                    uint32_t w[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) w[e] = __float_as_uint(acc[8 * j + e]);
+                    stg256(out + 8 * j, w);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    reinterpret_cast<float4*>(out)[j] =
+                        make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
+            }
         }
     }
     return true;

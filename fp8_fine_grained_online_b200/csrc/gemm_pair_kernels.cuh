@@ -43,8 +43,8 @@ constexpr uint64_t kDrainGraceNs = 2000000ull;            // abort path: let cop
 struct GemmPairSmemTail {
     uint64_t full[kPairStages];    // even CTA: TMA bytes of both CTAs
     uint64_t empty[kPairStages];   // both CTAs: MMA commit (multicast)
-    uint64_t tfull[4];             // both CTAs: MMA commit (multicast), per TMEM half-buffer
-    uint64_t tempty[4];            // even CTA: 16 epilogue-warp arrivals, per half-buffer
+    uint64_t tfull[2];             // both CTAs: MMA commit (multicast)
+    uint64_t tempty[2];            // even CTA: 16 epilogue-warp arrivals
     uint32_t tmem_base;
     int abort_flag;
     int total_tiles;
@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(&tail->full[s], 1);
             mbar_init(&tail->empty[s], 1);
         }
-        for (int b = 0; b < 4; ++b) {
+        for (int b = 0; b < 2; ++b) {
             mbar_init(&tail->tfull[b], 1);
             mbar_init(&tail->tempty[b], 2 * kEpiWarps);
         }
@@ -169,14 +169,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // two barrier waits, four UMMAs and two commits, against 512
             // cycles of tensor work; two threads keep the tensor pipe fed.
             const uint32_t par = warp == kMmaWarp ? 0u : 1u;
-            constexpr uint32_t idesc = idesc_e4m3_f32(kPairBM, kBN / 2);
+            constexpr uint32_t idesc = idesc_e4m3_f32(kPairBM, kBN);
             int stage = 0;
             uint32_t phase = 0;
             uint32_t chunk = 0;
             uint32_t last_issued = 0;
             bool issued_any = false;
-            int last_tfull = -1;          // last half-buffer committed, and its phase
-            uint32_t last_tfull_par = 0;
             bool ok = true;
             for (int t = pair; t < total_tiles && ok; t += num_pairs) {
                 for (int kb = 0; kb < nkb; ++kb) {
@@ -184,36 +182,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const uint32_t use = chunk >> 1;
                         // Operands first (usually long ready), then the TMEM
                         // buffer: the epilogue's release is the critical path.
-                        if (!bounded_wait(&tail->full[stage], phase, abort_flag)) {
+                        if (!bounded_wait(&tail->full[stage], phase, abort_flag) ||
+                            !bounded_wait(&tail->tempty[par], (use & 1u) ^ 1u, abort_flag)) {
                             ok = false;
                             break;
                         }
+                        tc_fence_after();
                         const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(stage_a(stage)));
-                        // Two UMMA halves of N = 128.  Half j reads B rows
-                        // [64 j, 64 j + 64) of each CTA's 128 (8 KB in), so its
-                        // 128 TMEM columns hold tile columns 64 j + [0, 64)
-                        // (even CTA's B) and 128 + 64 j + [0, 64) (odd CTA's).
+                        const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(stage_b(stage)));
+                        const uint32_t d = tmem_base + par * kBN;
 #pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            if (!bounded_wait(&tail->tempty[2 * par + j], (use & 1u) ^ 1u,
-                                              abort_flag)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
-                            const uint64_t bdesc =
-                                sdesc_kmajor_sw128(smem_u32(stage_b(stage) + j * (kPairHalfBytes / 2)));
-                            const uint32_t d = tmem_base + par * kBN + j * (kBN / 2);
-#pragma unroll
-                            for (int k = 0; k < kBK / 32; ++k)
-                                umma_f8f6f4_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc,
-                                                 k > 0 ? 1u : 0u);
-                            umma_commit_pair_mc(&tail->tfull[2 * par + j], 0x3);
-                            last_tfull = static_cast<int>(2 * par + j);
-                            last_tfull_par = use & 1u;
-                        }
-                        if (!ok) break;
+                        for (int k = 0; k < kBK / 32; ++k)
+                            umma_f8f6f4_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc,
+                                             k > 0 ? 1u : 0u);
                         umma_commit_pair_mc(&tail->empty[stage], 0x3);
+                        umma_commit_pair_mc(&tail->tfull[par], 0x3);
                         last_issued = chunk;
                         issued_any = true;
                     }
@@ -228,13 +211,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 // Both CTAs' epilogues release every buffer they used: wait for
                 // the last release of this issuer's buffer so that no remote
                 // arrival is in flight when the pair exits.
-                if (issued_any) {
-                    drain_wait(&tail->tempty[2 * par], (last_issued >> 1) & 1u);
-                    drain_wait(&tail->tempty[2 * par + 1], (last_issued >> 1) & 1u);
-                }
+                if (issued_any) drain_wait(&tail->tempty[par], (last_issued >> 1) & 1u);
             } else {
                 aborted = true;
-                if (last_tfull >= 0) drain_wait(&tail->tfull[last_tfull], last_tfull_par);
+                if (issued_any) drain_wait(&tail->tfull[par], (last_issued >> 1) & 1u);
             }
         }
     } else {
@@ -244,9 +224,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int h = warp >> 2;
         const int r = 128 * static_cast<int>(rank) + q * 32 + lane;   // row within the pair tile
         const uint32_t t_lane = static_cast<uint32_t>(q * 32) << 16;
-        uint32_t tempty_leader[4];
-#pragma unroll
-        for (int b = 0; b < 4; ++b) tempty_leader[b] = mapa_shared(smem_u32(&tail->tempty[b]), 0);
+        const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tail->tempty[0]), 0),
+                                           mapa_shared(smem_u32(&tail->tempty[1]), 0)};
         uint32_t chunk = 0;
         bool ok = true;
         for (int t = pair; t < total_tiles && ok; t += num_pairs) {
@@ -255,17 +234,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const bool row_ok = row < tc.row_end;
             const int64_t col0 = tc.n0 + h * 128;
             const bool col_ok = col0 < p.N;
-            ok = epilogue_tile<kOutBf16, kQuantOut, kColScaleB, true>(
+            ok = epilogue_tile<kOutBf16, kQuantOut, kColScaleB>(
                 p, tail->tfull, abort_flag, tmem_base, t_lane, h, lane, row, row_ok, col0, col_ok,
-                tc.g, chunk,
-                [&](uint32_t hb) {
-                    // hb is warp-uniform; selected without indexing registers
-                    uint32_t a = tempty_leader[0];
-#pragma unroll
-                    for (int b = 1; b < 4; ++b)
-                        if (hb == static_cast<uint32_t>(b)) a = tempty_leader[b];
-                    mbar_arrive_cluster(a);
-                },
+                tc.g, chunk, [&](uint32_t buf) { mbar_arrive_cluster(tempty_leader[buf]); },
                 sb_stages + warp * 2 * 128);
         }
         if (!ok) aborted = true;

@@ -21,11 +21,13 @@
 //   * every thread computes the block's scale and reciprocal and encodes its
 //     row with the FMA-corrected quotient (exact for bf16);
 //   * [K, N] output: the row's 128 codes leave as four 32-byte stores;
-//   * [N, K] output: the codes go through the slot just read (now free) as a
-//     word array U[g][k] (word g of row k = codes of columns 4g..4g+3,
+//   * the slot is refilled with the group's block kQwSlots ahead right after
+//     the group barrier (every row is in registers by then);
+//   * [N, K] output: the codes go through the group's 16 KB transpose buffer
+//     as a word array U[g][k] (word g of row k = codes of columns 4g..4g+3,
 //     16-byte chunks swizzled by g), then thread n gathers byte n % 4 of
 //     words U[n / 4][k] for every k (byte permutes) and writes output row n
-//     as four 32-byte stores.  The slot is refilled one block later.
+//     as four 32-byte stores.
 #pragma once
 
 #include <cstdint>
@@ -42,6 +44,7 @@ constexpr int kQwGroups = 2;                      // groups of 4 warps per CTA
 constexpr int kQwSlots = 3;
 constexpr int kQwHalfBytes = 128 * 128;           // 128 rows x 64 bf16
 constexpr int kQwBlockBytes = 2 * kQwHalfBytes;   // 32 KB: a 128x128 bf16 block
+constexpr int kQwTransposeBytes = 128 * 128;      // [N, K] output: 16 KB of codes per group
 constexpr int kQwThreads = kQwGroups * 128;
 
 struct QwSmemTail {
@@ -51,8 +54,9 @@ struct QwSmemTail {
     int abort_flag;
 };
 
-constexpr size_t kQwSmemBytes =
-    1024 /* alignment slack */ + kQwGroups * kQwSlots * kQwBlockBytes + sizeof(QwSmemTail);
+constexpr size_t kQwSmemBytes = 1024 /* alignment slack */ + kQwGroups * kQwSlots * kQwBlockBytes +
+                                kQwGroups * kQwTransposeBytes + sizeof(QwSmemTail);
+static_assert(kQwSmemBytes <= 227 * 1024, "shared memory per CTA");
 
 struct QwParams {
     int64_t nbr, nbc;          // blocks along K (rows of w) and N (columns)
@@ -85,8 +89,8 @@ __global__ void __launch_bounds__(kQwThreads, 1)
     quant_weight_rows_kernel(const __grid_constant__ CUtensorMap tm_in, const QwParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    QwSmemTail* tail =
-        reinterpret_cast<QwSmemTail*>(smem + kQwGroups * kQwSlots * kQwBlockBytes);
+    uint8_t* tbuf_base = smem + kQwGroups * kQwSlots * kQwBlockBytes;   // [N, K] output only
+    QwSmemTail* tail = reinterpret_cast<QwSmemTail*>(tbuf_base + kQwGroups * kQwTransposeBytes);
     volatile int* abort_flag = &tail->abort_flag;
 
     const int warp = threadIdx.x >> 5;
@@ -175,16 +179,8 @@ __global__ void __launch_bounds__(kQwThreads, 1)
                                     bf16x2_absmax(tail->red[g][par][2], tail->red[g][par][3]));
         bm &= 0x7FFF7FFFu;
         const float amax = fmaxf(__uint_as_float(bm << 16), __uint_as_float(bm & 0xFFFF0000u));
-        if (t == 0) {
-            if (!kTransposed) {
-                // [K, N]: the slot just read takes the block kQwSlots ahead.
-                if (k + kQwSlots < count) issue(k + kQwSlots);
-            } else if (k > 0 && k - 1 + kQwSlots < count) {
-                // [N, K]: the previous block's slot, whose transpose buffer
-                // every thread has finished reading (it passed this barrier).
-                issue(k - 1 + kQwSlots);
-            }
-        }
+        // The slot just read takes the block kQwSlots ahead.
+        if (t == 0 && k + kQwSlots < count) issue(k + kQwSlots);
 
         const int64_t br = c_br, bc = c_bc;
         advance(c_br, c_bc);
@@ -225,10 +221,13 @@ __global__ void __launch_bounds__(kQwThreads, 1)
                 stg256_cs(dst + 32 * q4, w);
             }
         } else {
-            // Codes word gi of row t (columns 4gi..4gi+3) -> U[gi][t].
+            // Codes word gi of row t (columns 4gi..4gi+3) -> U[gi][t], in the
+            // group's transpose buffer.  Every thread finished reading the
+            // previous block's U before it passed this block's first barrier.
+            const uint32_t u_base = smem_u32(tbuf_base + g * kQwTransposeBytes);
 #pragma unroll
             for (int gi = 0; gi < 32; ++gi)
-                asm volatile("st.shared.u32 [%0], %1;" ::"r"(qw_u_addr(slot_addr, gi, t)),
+                asm volatile("st.shared.u32 [%0], %1;" ::"r"(qw_u_addr(u_base, gi, t)),
                              "r"(codes[gi])
                              : "memory");
             if (!qw_group_sync(&tail->gbar[g], uses, lane, abort_flag)) break;
@@ -241,14 +240,11 @@ __global__ void __launch_bounds__(kQwThreads, 1)
             uint32_t out[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                const uint4 w = lds128_addr(qw_u_addr(slot_addr, gi, 4u * j));
+                const uint4 w = lds128_addr(qw_u_addr(u_base, gi, 4u * j));
                 const uint32_t lo = __byte_perm(w.x, w.y, pick);
                 const uint32_t hi = __byte_perm(w.z, w.w, pick);
                 out[j] = __byte_perm(lo, hi, 0x5410);
             }
-            // This thread's shared-memory accesses to the slot come before the
-            // TMA load that will refill it (issued after a later barrier).
-            fence_proxy_async_shared();
             uint8_t* dst = p.q + (bc * 128 + t) * p.ldq + br * 128;
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {

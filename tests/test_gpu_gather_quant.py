@@ -24,6 +24,24 @@ def test_gather_quant_matches_oracle(cuda_lib, orc, T, R, K, dtype):
     assert_scales_equal(sa.cpu().numpy(), sao)
 
 
+@pytest.mark.parametrize("offset", [0, 16])
+def test_gather_quant_both_bf16_paths(cuda_lib, orc, offset):
+    """bf16 codes written with 32-byte alignment take the one-row-per-thread
+    kernel (rows fetched by bulk copies); codes at a 16-byte offset take the
+    register kernel.  Both equal the oracle and write nothing outside q."""
+    T, R, K = 97, 333, 640
+    x = synth.act_input(T, K, 1.0, 1e-2, 100.0, 7, "cpu", torch.bfloat16, tensor_id=4)
+    rows = torch.randint(0, T, (R,), generator=torch.Generator().manual_seed(9), dtype=torch.int32)
+    qbuf = torch.full((R, K + 16 + offset), 0xCD, dtype=torch.uint8, device="cuda")
+    q = qbuf[:, offset:offset + K]
+    _, sa = cuda_lib.fp8_quantize_act_1x128_gather(x.cuda(), rows.cuda(), q=q)
+    qo, sao = orc.quantize_act_1x128(to_oracle(x[rows.long()]))
+    assert_codes_equal(np_u8(q), qo)
+    assert_scales_equal(sa.cpu().numpy(), sao)
+    rest = np_u8(qbuf)
+    assert np.all(rest[:, :offset] == 0xCD) and np.all(rest[:, offset + K:] == 0xCD)
+
+
 def test_gather_quant_equals_gather_then_quantize(cuda_lib):
     d = synth.moe_inputs("cpu", tokens=1024, experts=32, with_weights=False)
     x = synth.act_input(1024, 7168, 1.0, 1e-3, 100.0, synth.MOE.config_id, "cpu").cuda()

@@ -109,6 +109,26 @@ def test_gemm_strided_output_and_operands(cuda_lib, orc):
     assert np.all(rest[:, :32] == 7.0) and np.all(rest[:, 32 + N:] == 7.0)
 
 
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_gemm_output_store_paths_agree(cuda_lib, orc, out_dtype):
+    """C with 32-byte aligned rows is written as 32-byte stores, C at a
+    16-byte offset as 16-byte stores: the two outputs are bit-identical and
+    within the bound, and nothing outside C is written."""
+    M, N, K = 300, 512, 640
+    qa, sa, qb, sb = oracle_operands(orc, M, N, K, 17)
+    args = (cuda_u8(qa), torch.from_numpy(sa).cuda(), cuda_u8(qb), torch.from_numpy(sb).cuda())
+    c_al = cuda_lib.fp8_blockscaled_gemm(*args, out_dtype=out_dtype)
+    off = 16 // c_al.element_size()
+    cbuf = torch.full((M, N + 2 * off), 3.0, dtype=out_dtype, device="cuda")
+    c_un = cbuf[:, off:off + N]
+    cuda_lib.fp8_blockscaled_gemm(*args, c=c_un)
+    assert torch.equal(c_al, c_un)
+    C_ref, T = orc.gemm_ref(qa, sa, qb, sb)
+    assert_gemm_within_bound(np_f32(c_un), C_ref, T, out_dtype)
+    rest = np_f32(cbuf)
+    assert np.all(rest[:, :off] == 3.0) and np.all(rest[:, off + N:] == 3.0)
+
+
 def test_gemm_degenerate_sizes(cuda_lib):
     dev = "cuda"
     a = torch.zeros((0, 128), dtype=torch.uint8, device=dev)
