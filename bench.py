@@ -714,7 +714,7 @@ class MoE(Workload):
     dominant = "grouped_gemm_gate_up"
 
     def __init__(self, fp8, device, tokens=8192, experts=256, topk=8, hidden=7168, inter=2048,
-                 dispatch="gather"):
+                 dispatch="scatter"):
         self.fp8 = fp8
         self.T, self.E, self.k, self.H, self.I = tokens, experts, topk, hidden, inter
         self.R = tokens * topk
@@ -1060,7 +1060,7 @@ def main():
                     help="comma list of workloads timed after the headline and reported under "
                          "'workloads' (default: all others when the headline is ffn; 'none')")
     ap.add_argument("--no-quant-error", action="store_true")
-    ap.add_argument("--moe-dispatch", choices=["gather", "scatter"], default="gather",
+    ap.add_argument("--moe-dispatch", choices=["gather", "scatter"], default="scatter",
                     help="MoE workload only: dispatch in row order (gather) or token order")
     ap.add_argument("--moe-experts", type=int, default=256,
                     help="MoE workload only: number of experts (tokens = 32 x experts)")

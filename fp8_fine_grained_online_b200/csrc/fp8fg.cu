@@ -9,7 +9,6 @@
 
 #include <atomic>
 #include <cstdint>
-#include <cstring>
 #include <mutex>
 
 #include "../../include/fp8fg.h"
@@ -92,12 +91,11 @@ fp8_status_t current_device(int* dev_out, int* sms_out) {
                 const void* qa_kernels[] = {
                     reinterpret_cast<const void*>(&quant_act_rows_kernel<kRowsPlain>),
                     reinterpret_cast<const void*>(&quant_act_rows_kernel<kRowsScatter>),
-                    reinterpret_cast<const void*>(&quant_act_rows_kernel<kRowsGather>),
                     reinterpret_cast<const void*>(&quant_weight_rows_kernel<false>),
                     reinterpret_cast<const void*>(&quant_weight_rows_kernel<true>)};
-                const size_t qa_bytes[] = {kQaSmemBytes, kQaSmemBytes, kQaSmemBytes,
-                                           kQwSmemBytes, kQwSmemBytes};
-                for (int i = 0; i < 5; ++i) {
+                const size_t qa_bytes[] = {kQaSmemBytes, kQaSmemBytes, kQwSmemBytes,
+                                           kQwSmemBytes};
+                for (int i = 0; i < 4; ++i) {
                     if (cudaFuncSetAttribute(qa_kernels[i],
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(qa_bytes[i])) != cudaSuccess) {
@@ -343,30 +341,6 @@ fp8_status_t launch_quant_act_rows(const void* x, int64_t M, int64_t K, int64_t 
     return launch_status();
 }
 
-// Gather form: output row r <- bf16 input row rows[r] of x [src_rows, ldx],
-// fetched row by row with bulk copies (no tensor map).
-fp8_status_t launch_quant_act_rows_gather(const void* x, int64_t src_rows, int64_t K, int64_t ldx,
-                                          const int32_t* rows, int64_t R, uint8_t* q,
-                                          int64_t ldq, float* sa, int64_t sa_stride_m,
-                                          int64_t sa_stride_kb, int sms, cudaStream_t stream) {
-    CUtensorMap unused;
-    memset(&unused, 0, sizeof unused);
-    QaParams p{};
-    p.rows = R;
-    p.nkb = K / 128;
-    p.nboxes = ((R + kQaRows - 1) / kQaRows) * p.nkb;
-    p.q = q; p.ldq = ldq;
-    p.s = sa; p.s_stride_m = sa_stride_m; p.s_stride_kb = sa_stride_kb;
-    p.gidx = rows;
-    p.x = static_cast<const uint16_t*>(x);
-    p.ldx = ldx;
-    p.src_rows = src_rows;
-    const int64_t ctas = (p.nboxes + kQaWarps - 1) / kQaWarps;
-    const unsigned grid = static_cast<unsigned>(ctas < sms ? ctas : sms);
-    quant_act_rows_kernel<kRowsGather><<<grid, kQaThreads, kQaSmemBytes, stream>>>(unused, p);
-    return launch_status();
-}
-
 template <typename T, int kMode>
 fp8_status_t launch_quant_stream_t(const CUtensorMap& map, const QsParams& p, int sms,
                                    cudaStream_t stream) {
@@ -509,12 +483,6 @@ fp8_status_t fp8_quantize_act_1x128_gather(const void* x, fp8_in_t x_type, int64
     int dev, sms;
     fp8_status_t st = current_device(&dev, &sms);
     if (st != FP8_OK) return st;
-    // bf16 rows whose codes can leave as 32-byte stores: one row per thread,
-    // rows fetched by bulk copies.
-    if (x_type == FP8_IN_BF16 && aligned32(q) && ldq % 32 == 0 && src_rows <= INT32_MAX &&
-        R <= INT32_MAX)
-        return launch_quant_act_rows_gather(x, src_rows, K, ldx, rows, R, q, ldq, sa, sa_stride_m,
-                                            sa_stride_kb, sms, stream);
     // one half-warp per output row at a time
     const int64_t grid = grid_for((R + 15) / 16, sms, kGqMinBlocks);
     const unsigned g = static_cast<unsigned>(grid);

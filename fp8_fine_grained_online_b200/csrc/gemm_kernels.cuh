@@ -77,6 +77,34 @@ __device__ __forceinline__ void record_device_error(unsigned code) {
     atomicCAS(&g_device_error, 0u, code);
 }
 
+// The limit of the waits that can abort (bounded_wait) is a device variable,
+// kWaitLimitCycles unless fp8_set_wait_limit() changed it.  Each CTA copies it
+// into shared memory at start (WaitCtl, next to its abort flag), so that no
+// wait depends on a global load.  A limit below kShortWaitLimit is a test of
+// the timeout path: the waits then check the clock after every poll instead
+// of every kPollsPerClockCheck polls, so that a real wait runs out.  The
+// drains below always keep kWaitLimitCycles.
+constexpr long long kWaitLimitCycles = 1ll << 31;
+constexpr long long kShortWaitLimit = 1ll << 20;
+constexpr int kPollsPerClockCheck = 64;
+
+__device__ long long g_wait_limit_cycles = kWaitLimitCycles;
+
+// A CTA's abort flag and its copy of the wait limit.  The flag is the first
+// member: the waits receive a pointer to it.
+struct WaitCtl {
+    int abort_flag;
+    int polls_per_check;
+    long long limit;
+};
+
+__device__ __forceinline__ void init_wait_ctl(WaitCtl* w) {
+    const long long limit = *static_cast<volatile long long*>(&g_wait_limit_cycles);
+    w->abort_flag = 0;
+    w->limit = limit;
+    w->polls_per_check = limit < kShortWaitLimit ? 1 : kPollsPerClockCheck;
+}
+
 struct GemmParams {
     const float* sa;
     int64_t sa_sm, sa_skb;
@@ -124,9 +152,8 @@ struct GemmSmemTail {
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint32_t tmem_base;
-    int abort_flag;
     int total_tiles;
-    int pad;
+    WaitCtl wait;
     GroupTables grp;
 };
 
@@ -146,39 +173,36 @@ struct TileCoord {
 // counter; the device-wide %globaltimer is slow to read and would delay the
 // reaction to a completed barrier).  2^31 cycles is about one second at the
 // B200's 1.9 GHz and a few seconds at its lowest clocks.
-// The limit of the waits that can abort (bounded_wait) is read from a device
-// variable, kWaitLimitCycles unless fp8_set_wait_limit() changed it: a test
-// shortens it to make real waits run out and exercise the abort path.  The
-// drains below always keep kWaitLimitCycles.
-constexpr long long kWaitLimitCycles = 1ll << 31;
-constexpr int kPollsPerClockCheck = 64;
-constexpr int kFastPolls = 16;
-
-__device__ long long g_wait_limit_cycles = kWaitLimitCycles;
-
+// The normal form polls kPollsPerClockCheck times (unrolled) between checks
+// of the abort flag and the clock: measured, any extra work in the polling
+// loop (a loop counter, a clock read per poll) slows the GEMM by 6-20%,
+// because spinning warps share issue slots with the epilogue.  The test form
+// (a limit below kShortWaitLimit) checks after every poll.
 __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity,
                                              volatile int* abort_flag) {
     const uint32_t a = smem_u32(bar);
+    const volatile WaitCtl* ctl = reinterpret_cast<const volatile WaitCtl*>(abort_flag);
+    const bool every_poll = ctl->polls_per_check == 1;   // read before the first poll
     if (mbar_try_wait(a, parity)) return true;
     const long long t0 = clock64();
-    // Fast path: most waits end within a few polls, and nothing here may
-    // wait on a memory load (the reaction to a completed phase is on the
-    // critical path of the GEMM pipeline).
-#pragma unroll 1
-    for (int i = 0; i < kFastPolls; ++i)
-        if (mbar_try_wait(a, parity)) return true;
-    // Slow path: the limit (constant while any kernel runs), the clock every
-    // poll, the CTA's abort flag every kPollsPerClockCheck polls.
-    const long long limit = __ldg(&g_wait_limit_cycles);
-    for (int i = 1;; ++i) {
-        if (mbar_try_wait(a, parity)) return true;
-        if (i % kPollsPerClockCheck == 0 && *abort_flag) return false;
-        if (clock64() - t0 > limit) {
-            *abort_flag = 1;
-            record_device_error(kDevErrTimeout);
-            return false;
+    if (!every_poll) {
+        while (true) {
+#pragma unroll
+            for (int i = 0; i < kPollsPerClockCheck; ++i)
+                if (mbar_try_wait(a, parity)) return true;
+            if (*abort_flag) return false;
+            if (clock64() - t0 > ctl->limit) break;
+        }
+    } else {
+        while (true) {
+            if (mbar_try_wait(a, parity)) return true;
+            if (*abort_flag) return false;
+            if (clock64() - t0 > ctl->limit) break;
         }
     }
+    *abort_flag = 1;
+    record_device_error(kDevErrTimeout);
+    return false;
 }
 
 // bounded_wait by every lane of a converged warp, decided for the warp as a
@@ -531,7 +555,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint8_t* sA = smem;                         // kStages x 16 KB
     uint8_t* sB = smem + kStages * kABytes;     // kStages x 32 KB
     GemmSmemTail* tail = reinterpret_cast<GemmSmemTail*>(smem + kStages * kStageBytes);
-    volatile int* abort_flag = &tail->abort_flag;
+    volatile int* abort_flag = &tail->wait.abort_flag;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -545,7 +569,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(&tail->tfull[b], 1);
             mbar_init(&tail->tempty[b], kEpiWarps);
         }
-        tail->abort_flag = 0;
+        init_wait_ctl(&tail->wait);
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);

@@ -46,9 +46,9 @@ struct GemmPairSmemTail {
     uint64_t tfull[2];             // both CTAs: MMA commit (multicast)
     uint64_t tempty[2];            // even CTA: 16 epilogue-warp arrivals
     uint32_t tmem_base;
-    int abort_flag;
     int total_tiles;
-    int pad;
+    WaitCtl wait;
+    uint64_t pad;                  // 16-byte multiple
 };
 
 constexpr size_t kGemmPairSmemBytes =
@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         reinterpret_cast<GemmPairSmemTail*>(smem + kPairStages * kPairStageBytes);
     GroupTables* gt = reinterpret_cast<GroupTables*>(tail + 1);   // grouped only
     float* sb_stages = reinterpret_cast<float*>(tail + 1);         // per-column sb only
-    volatile int* abort_flag = &tail->abort_flag;
+    volatile int* abort_flag = &tail->wait.abort_flag;
     auto stage_a = [&](int s) { return smem + s * kPairStageBytes; };
     auto stage_b = [&](int s) { return smem + s * kPairStageBytes + kPairHalfBytes; };
 
@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(&tail->tfull[b], 1);
             mbar_init(&tail->tempty[b], 2 * kEpiWarps);
         }
-        tail->abort_flag = 0;
+        init_wait_ctl(&tail->wait);
         if (!kGrouped) tail->total_tiles = p.num_mt * p.num_nt;
         fence_mbar_init();
         tma_prefetch_desc(&tmA);

@@ -49,21 +49,14 @@ constexpr int kQaThreads = 32 * kQaWarps;
 enum QaMode {
     kRowsPlain = 0,    // input row m -> output row m
     kRowsScatter = 1,  // input row t (a token) -> output rows dest[t, :]
-    kRowsGather = 2,   // input row rows[r] -> output row r
 };
-// The gather form fills a box row by row (one 256-byte bulk copy per lane)
-// into rows 272 bytes apart: the 16-byte pad puts chunk c of 8 consecutive
-// rows in 8 distinct bank groups.
-constexpr int kQaGatherRowBytes = 256 + 16;
-constexpr int kQaGatherBoxBytes = kQaRows * kQaGatherRowBytes;
 
 struct QaSmemTail {
     uint64_t full[kQaWarps][kQaSlots];
-    int abort_flag;
+    WaitCtl wait;
 };
 
-constexpr int kQaRingBytes = kQaWarps * kQaSlots *
-                             (kQaGatherBoxBytes > kQaBoxBytes ? kQaGatherBoxBytes : kQaBoxBytes);
+constexpr int kQaRingBytes = kQaWarps * kQaSlots * kQaBoxBytes;
 constexpr size_t kQaSmemBytes = 1024 /* alignment slack */ + kQaRingBytes + sizeof(QaSmemTail);
 static_assert(kQaSmemBytes <= 227 * 1024, "shared memory per CTA");
 
@@ -80,25 +73,7 @@ struct QaParams {
     const int32_t* dest;
     int64_t topk;
     int64_t out_rows;
-    // Gather form: output row r (of rows) is input row gidx[r] of x
-    // [src_rows, ldx] (bf16).
-    const int32_t* gidx;
-    const uint16_t* x;
-    int64_t ldx;
-    int64_t src_rows;
 };
-
-// Bulk copy (no tensor map) of `bytes` from global to this CTA's shared
-// memory, completion counted in bytes on `bar`.  Both addresses 16-byte
-// aligned, bytes a multiple of 16.
-__device__ __forceinline__ void bulk_load_g2s(uint32_t dst, const void* src, uint32_t bytes,
-                                              uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-            "r"(dst),
-        "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
-}
 
 // max(|a|, |b|) per bf16 lane (sign bits are the XOR of the inputs' and are
 // cleared by the caller); a NaN lane yields the other operand.
@@ -137,30 +112,27 @@ __device__ __forceinline__ void store_row_tile(const QaParams& p, int64_t row, i
     p.s[row * p.s_stride_m + kb * p.s_stride_kb] = s;
 }
 
-// kMode (QaMode): plain rows; or the MoE dispatch fused in, in token order
+// kMode (QaMode): plain rows, or the MoE dispatch fused in, in token order
 // (scatter: each token row is read and quantized once, and its codes and
-// scale are written to each of its up to topk destination rows) or in row
-// order (gather: output row r is filled from input row gidx[r]; the rows of a
-// box are fetched by per-row bulk copies instead of TMA tiles).
+// scale are written to each of its up to topk destination rows).
 template <int kMode>
 __global__ void __launch_bounds__(kQaThreads, 1)
     quant_act_rows_kernel(const __grid_constant__ CUtensorMap tm_in, const QaParams p) {
     constexpr bool kScatter = kMode == kRowsScatter;
-    constexpr bool kGather = kMode == kRowsGather;
-    constexpr int kSlotBytes = kGather ? kQaGatherBoxBytes : kQaBoxBytes;
+    constexpr int kSlotBytes = kQaBoxBytes;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     QaSmemTail* tail = reinterpret_cast<QaSmemTail*>(smem + kQaRingBytes);
-    volatile int* abort_flag = &tail->abort_flag;
+    volatile int* abort_flag = &tail->wait.abort_flag;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int w = 0; w < kQaWarps; ++w)
             for (int s = 0; s < kQaSlots; ++s) mbar_init(&tail->full[w][s], 1);
-        tail->abort_flag = 0;
+        init_wait_ctl(&tail->wait);
         fence_mbar_init();
-        if (!kGather) tma_prefetch_desc(&tm_in);
+        tma_prefetch_desc(&tm_in);
     }
     __syncthreads();
 
@@ -198,59 +170,20 @@ __global__ void __launch_bounds__(kQaThreads, 1)
         tma_load_2d(dst + kQaHalfBytes, &tm_in, &full[slot], x + 64, y);
         advance(i_mb, i_kb);
     };
-    // Gather form: the whole warp issues box k; lane r copies the 256 bytes
-    // of tile i_kb of input row `src` (its output row's gather index, already
-    // loaded) when that index is valid.  valid_bits keeps, per slot, whether
-    // this lane's row of the box was fetched.
-    uint32_t valid_bits = 0;
-    auto gather_index = [&]() -> int32_t {   // index of this lane's row of the next box to issue
-        const int64_t r = i_mb * kQaRows + lane;
-        return r < p.rows ? __ldg(p.gidx + r) : -1;
-    };
-    auto issue_gather = [&](int64_t k, int32_t src) {
-        const int slot = static_cast<int>(k % kQaSlots);
-        const int64_t r = i_mb * kQaRows + lane;
-        const bool valid = r < p.rows && src >= 0 && src < p.src_rows;
-        if (r < p.rows && !valid && i_kb == 0) record_device_error(kDevErrShape);
-        const unsigned vmask = __ballot_sync(0xFFFFFFFFu, valid);
-        if (lane == 0) mbar_arrive_expect_tx(&full[slot], 256u * __popc(vmask));
-        __syncwarp();
-        if (valid)
-            bulk_load_g2s(smem_u32(ring + slot * kSlotBytes + lane * kQaGatherRowBytes),
-                          p.x + src * p.ldx + i_kb * 128, 256, smem_u32(&full[slot]));
-        valid_bits = (valid_bits & ~(1u << slot)) | (valid ? 1u << slot : 0u);
-        advance(i_mb, i_kb);
-    };
-    if constexpr (kGather) {
-        for (int64_t k = 0; k < kQaSlots && k < count; ++k) issue_gather(k, gather_index());
-    } else if (lane == 0) {
+    if (lane == 0)
         for (int64_t k = 0; k < kQaSlots && k < count; ++k) issue(k);
-    }
 
     const uint32_t swz = static_cast<uint32_t>(lane & 7);
     for (int64_t k = 0; k < count; ++k) {
         const int slot = static_cast<int>(k % kQaSlots);
         if (!bounded_wait_warp(&full[slot], static_cast<uint32_t>((k / kQaSlots) & 1), abort_flag))
             break;
-        // Gather form: the index of the box this iteration will issue, loaded
-        // now so that its latency hides behind the loads and the amax.
-        int32_t next_src = -1;
-        if constexpr (kGather) {
-            if (k + kQaSlots < count) next_src = gather_index();
-        }
-        const bool row_valid = !kGather || ((valid_bits >> slot) & 1u);
         Raw8<uint16_t> raw[16];
-        if constexpr (kGather) {
-            const uint32_t row_addr = smem_u32(ring + slot * kSlotBytes) + lane * kQaGatherRowBytes;
+        const uint32_t row_addr = smem_u32(ring + slot * kSlotBytes) + lane * 128;
 #pragma unroll
-            for (int c = 0; c < 16; ++c) raw[c].a = lds128_addr(row_addr + c * 16);
-        } else {
-            const uint32_t row_addr = smem_u32(ring + slot * kSlotBytes) + lane * 128;
-#pragma unroll
-            for (int c = 0; c < 16; ++c)
-                raw[c].a = lds128_addr(row_addr + (c >> 3) * kQaHalfBytes +
-                                       (((static_cast<uint32_t>(c) & 7u) ^ swz) << 4));
-        }
+        for (int c = 0; c < 16; ++c)
+            raw[c].a = lds128_addr(row_addr + (c >> 3) * kQaHalfBytes +
+                                   (((static_cast<uint32_t>(c) & 7u) ^ swz) << 4));
         // amax of the row's 128 values: packed |max| over the 64 pairs.
         uint32_t m[16];
 #pragma unroll
@@ -265,11 +198,7 @@ __global__ void __launch_bounds__(kQaThreads, 1)
         const float amax = fmaxf(__uint_as_float(mm << 16), __uint_as_float(mm & 0xFFFF0000u));
         // Every lane's row is in registers: the slot takes the box kQaSlots on.
         __syncwarp();
-        if constexpr (kGather) {
-            if (k + kQaSlots < count) issue_gather(k + kQaSlots, next_src);
-        } else if (lane == 0 && k + kQaSlots < count) {
-            issue(k + kQaSlots);
-        }
+        if (lane == 0 && k + kQaSlots < count) issue(k + kQaSlots);
 
         const int64_t kb = c_kb;
         const int64_t row = c_mb * kQaRows + lane;
@@ -327,7 +256,7 @@ __global__ void __launch_bounds__(kQaThreads, 1)
                     store_row_tile(p, d, kb, codes, s);
                 }
             }
-        } else if (row < p.rows && row_valid) {
+        } else if (row < p.rows) {
             store_row_tile(p, row, kb, codes, s);
         }
     }

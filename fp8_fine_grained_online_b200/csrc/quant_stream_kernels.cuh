@@ -66,7 +66,7 @@ struct alignas(16) QsSmemTail {
     uint64_t full[kQsMaxStages];       // slot filled (TMA bytes)
     uint64_t gbar[kQsGroups];          // per-group barrier (8 warp arrivals)
     float red[kQsGroups][2][8];        // [group][block parity][warp]
-    int abort_flag;
+    WaitCtl wait;
 };
 
 // Transposed output only: [group][box parity][n][k/4 swizzled], transposed
@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kQsThreads, 1)
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     QsSmemTail* tail = reinterpret_cast<QsSmemTail*>(smem + kStages * kBoxBytes);
     QsTransposeBuf* tx = reinterpret_cast<QsTransposeBuf*>(tail + 1);   // [N, K] output only
-    volatile int* abort_flag = &tail->abort_flag;
+    volatile int* abort_flag = &tail->wait.abort_flag;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -189,7 +189,7 @@ __global__ void __launch_bounds__(kQsThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) mbar_init(&tail->full[s], 1);
         for (int gi = 0; gi < kQsGroups; ++gi) mbar_init(&tail->gbar[gi], 8);
-        tail->abort_flag = 0;
+        init_wait_ctl(&tail->wait);
         fence_mbar_init();
         tma_prefetch_desc(&tm_in);
     }

@@ -51,7 +51,7 @@ struct QwSmemTail {
     uint64_t full[kQwGroups][kQwSlots];   // slot filled (TMA bytes)
     uint64_t gbar[kQwGroups];             // group barrier: 4 warp arrivals
     uint32_t red[kQwGroups][2][4];        // per warp packed |max|, by block parity
-    int abort_flag;
+    WaitCtl wait;
 };
 
 constexpr size_t kQwSmemBytes = 1024 /* alignment slack */ + kQwGroups * kQwSlots * kQwBlockBytes +
@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(kQwThreads, 1)
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* tbuf_base = smem + kQwGroups * kQwSlots * kQwBlockBytes;   // [N, K] output only
     QwSmemTail* tail = reinterpret_cast<QwSmemTail*>(tbuf_base + kQwGroups * kQwTransposeBytes);
-    volatile int* abort_flag = &tail->abort_flag;
+    volatile int* abort_flag = &tail->wait.abort_flag;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(kQwThreads, 1)
             for (int s = 0; s < kQwSlots; ++s) mbar_init(&tail->full[gi][s], 1);
             mbar_init(&tail->gbar[gi], 4);
         }
-        tail->abort_flag = 0;
+        init_wait_ctl(&tail->wait);
         fence_mbar_init();
         tma_prefetch_desc(&tm_in);
     }

@@ -26,9 +26,8 @@ def test_gather_quant_matches_oracle(cuda_lib, orc, T, R, K, dtype):
 
 @pytest.mark.parametrize("offset", [0, 16])
 def test_gather_quant_both_bf16_paths(cuda_lib, orc, offset):
-    """bf16 codes written with 32-byte alignment take the one-row-per-thread
-    kernel (rows fetched by bulk copies); codes at a 16-byte offset take the
-    register kernel.  Both equal the oracle and write nothing outside q."""
+    """Codes at 32-byte and 16-byte offsets: both equal the oracle and nothing
+    outside q is written."""
     T, R, K = 97, 333, 640
     x = synth.act_input(T, K, 1.0, 1e-2, 100.0, 7, "cpu", torch.bfloat16, tensor_id=4)
     rows = torch.randint(0, T, (R,), generator=torch.Generator().manual_seed(9), dtype=torch.int32)
