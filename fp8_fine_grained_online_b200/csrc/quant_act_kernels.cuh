@@ -173,6 +173,21 @@ __global__ void __launch_bounds__(kQaThreads, 1)
     if (lane == 0)
         for (int64_t k = 0; k < kQaSlots && k < count; ++k) issue(k);
 
+    // Scatter form: the first kDestBatch destinations of this lane's token,
+    // for the box being processed (dst_cur) and, fetched one box ahead so
+    // that the loads' latency hides behind a whole box, the next (dst_next).
+    constexpr int kDestBatch = 8;
+    int32_t dst_cur[kDestBatch], dst_next[kDestBatch];
+    auto load_dest = [&](int64_t mb, int32_t (&d)[kDestBatch]) {
+        const int64_t row = mb * kQaRows + lane;
+#pragma unroll
+        for (int j = 0; j < kDestBatch; ++j)
+            d[j] = (row < p.rows && j < p.topk) ? __ldg(p.dest + row * p.topk + j) : -1;
+    };
+    if constexpr (kScatter) {
+        if (count > 0) load_dest(c_mb, dst_cur);
+    }
+
     const uint32_t swz = static_cast<uint32_t>(lane & 7);
     for (int64_t k = 0; k < count; ++k) {
         const int slot = static_cast<int>(k % kQaSlots);
@@ -203,13 +218,8 @@ __global__ void __launch_bounds__(kQaThreads, 1)
         const int64_t kb = c_kb;
         const int64_t row = c_mb * kQaRows + lane;
         advance(c_mb, c_kb);
-        // Scatter form: the row's first destinations, fetched while it encodes.
-        constexpr int kDestBatch = 8;
-        int32_t dst_rows[kDestBatch];
         if constexpr (kScatter) {
-#pragma unroll
-            for (int j = 0; j < kDestBatch; ++j)
-                dst_rows[j] = (row < p.rows && j < p.topk) ? __ldg(p.dest + row * p.topk + j) : -1;
+            if (k + 1 < count) load_dest(c_mb, dst_next);   // c_mb is now the next box's band
         }
         const float s = scale_from_amax(amax);
         const float r = __frcp_rn(s);
@@ -238,13 +248,13 @@ __global__ void __launch_bounds__(kQaThreads, 1)
         }
         if constexpr (kScatter) {
             for (int64_t j0 = 0; j0 < p.topk; j0 += kDestBatch) {
-                if (j0 > 0) {
+                int32_t dst_rows[kDestBatch];
 #pragma unroll
-                    for (int j = 0; j < kDestBatch; ++j)
-                        dst_rows[j] = (row < p.rows && j0 + j < p.topk)
-                                          ? __ldg(p.dest + row * p.topk + j0 + j)
-                                          : -1;
-                }
+                for (int j = 0; j < kDestBatch; ++j)
+                    dst_rows[j] = j0 == 0 ? dst_cur[j]
+                                  : (row < p.rows && j0 + j < p.topk)
+                                      ? __ldg(p.dest + row * p.topk + j0 + j)
+                                      : -1;
 #pragma unroll
                 for (int j = 0; j < kDestBatch; ++j) {
                     const int32_t d = dst_rows[j];
@@ -256,6 +266,8 @@ __global__ void __launch_bounds__(kQaThreads, 1)
                     store_row_tile(p, d, kb, codes, s);
                 }
             }
+#pragma unroll
+            for (int j = 0; j < kDestBatch; ++j) dst_cur[j] = dst_next[j];
         } else if (row < p.rows) {
             store_row_tile(p, row, kb, codes, s);
         }

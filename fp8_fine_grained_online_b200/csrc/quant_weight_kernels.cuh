@@ -13,21 +13,22 @@
 // kQwSlots shared-memory slots (32 KB each):
 //   * the group's first thread fills a slot with two TMA loads of 128 rows x
 //     64 bf16 (128-byte swizzle: 16-byte chunk c of row r sits at chunk
-//     c ^ (r % 8), so 8 lanes reading chunk c of 8 consecutive rows hit 8
-//     distinct bank groups);
-//   * thread t of the group takes block row t into 64 registers, reduces it
+//     c ^ (r % 8));
+//   * each thread takes its share of the block into registers, reduces it
 //     with packed |max|, and the warp and then the group (through shared
-//     memory and a bounded group barrier) combine the block's amax;
+//     memory and a bounded group barrier) combine the block's amax; the slot
+//     is refilled with the group's block kQwSlots ahead right after that
+//     barrier (every value is in registers by then);
 //   * every thread computes the block's scale and reciprocal and encodes its
-//     row with the FMA-corrected quotient (exact for bf16);
-//   * [K, N] output: the row's 128 codes leave as four 32-byte stores;
-//   * the slot is refilled with the group's block kQwSlots ahead right after
-//     the group barrier (every row is in registers by then);
-//   * [N, K] output: the codes go through the group's 16 KB transpose buffer
-//     as a word array U[g][k] (word g of row k = codes of columns 4g..4g+3,
-//     16-byte chunks swizzled by g), then thread n gathers byte n % 4 of
-//     words U[n / 4][k] for every k (byte permutes) and writes output row n
-//     as four 32-byte stores.
+//     values with the FMA-corrected quotient (exact for bf16).
+// [K, N] output: thread t holds block row t (16 x 16-byte loads: 8 lanes
+// read chunk c of 8 consecutive rows, 8 distinct bank groups) and writes its
+// 128 codes as four 32-byte stores.
+// [N, K] output: thread t holds the column pair 2cp, 2cp+1 (cp = t % 64) over
+// block rows 64 kh .. 64 kh + 63 (kh = t / 64): 64 four-byte loads, a warp
+// reading one whole 128-byte row per load (no bank conflict).  The low and
+// high halves of its words are two rows of the transposed output; each gets
+// 64 codes, two 32-byte stores.  No transpose buffer, one barrier per block.
 #pragma once
 
 #include <cstdint>
@@ -44,7 +45,6 @@ constexpr int kQwGroups = 2;                      // groups of 4 warps per CTA
 constexpr int kQwSlots = 3;
 constexpr int kQwHalfBytes = 128 * 128;           // 128 rows x 64 bf16
 constexpr int kQwBlockBytes = 2 * kQwHalfBytes;   // 32 KB: a 128x128 bf16 block
-constexpr int kQwTransposeBytes = 128 * 128;      // [N, K] output: 16 KB of codes per group
 constexpr int kQwThreads = kQwGroups * 128;
 
 struct QwSmemTail {
@@ -54,8 +54,8 @@ struct QwSmemTail {
     WaitCtl wait;
 };
 
-constexpr size_t kQwSmemBytes = 1024 /* alignment slack */ + kQwGroups * kQwSlots * kQwBlockBytes +
-                                kQwGroups * kQwTransposeBytes + sizeof(QwSmemTail);
+constexpr size_t kQwSmemBytes =
+    1024 /* alignment slack */ + kQwGroups * kQwSlots * kQwBlockBytes + sizeof(QwSmemTail);
 static_assert(kQwSmemBytes <= 227 * 1024, "shared memory per CTA");
 
 struct QwParams {
@@ -78,19 +78,13 @@ __device__ __forceinline__ bool qw_group_sync(uint64_t* bar, uint32_t& uses, int
     return ok;
 }
 
-// Shared word address of U[g][k] in a slot: row g (512 bytes) of 128 words,
-// 16-byte chunk (k / 4) stored at chunk (k / 4) ^ (g % 8).
-__device__ __forceinline__ uint32_t qw_u_addr(uint32_t base, uint32_t g, uint32_t k) {
-    return base + g * 512u + ((((k >> 2) ^ (g & 7u)) << 4) | ((k & 3u) << 2));
-}
-
 template <bool kTransposed>
 __global__ void __launch_bounds__(kQwThreads, 1)
     quant_weight_rows_kernel(const __grid_constant__ CUtensorMap tm_in, const QwParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint8_t* tbuf_base = smem + kQwGroups * kQwSlots * kQwBlockBytes;   // [N, K] output only
-    QwSmemTail* tail = reinterpret_cast<QwSmemTail*>(tbuf_base + kQwGroups * kQwTransposeBytes);
+    QwSmemTail* tail =
+        reinterpret_cast<QwSmemTail*>(smem + kQwGroups * kQwSlots * kQwBlockBytes);
     volatile int* abort_flag = &tail->wait.abort_flag;
 
     const int warp = threadIdx.x >> 5;
@@ -146,22 +140,47 @@ __global__ void __launch_bounds__(kQwThreads, 1)
         for (int64_t k = 0; k < kQwSlots && k < count; ++k) issue(k);
 
     const uint32_t swz = static_cast<uint32_t>(t & 7);
+    // [N, K] output: thread t holds the column pair cp = t % 64 (columns 2cp,
+    // 2cp + 1 of the block) over the block rows kh * 64 .. kh * 64 + 63.
+    const uint32_t cp = static_cast<uint32_t>(t) & 63u;
+    const uint32_t kh = static_cast<uint32_t>(t) >> 6;
     for (int64_t k = 0; k < count; ++k) {
         const int slot = static_cast<int>(k % kQwSlots);
         if (!bounded_wait_warp(&full[slot], static_cast<uint32_t>((k / kQwSlots) & 1), abort_flag))
             break;
         const uint32_t slot_addr = smem_u32(ring + slot * kQwBlockBytes);
-        const uint32_t row_addr = slot_addr + t * 128;
+        // kTransposed: w2[i] = (w[k][2cp], w[k][2cp+1]) for k = 64 kh + i, a
+        // 4-byte load from the swizzled box (the 32 lanes of a warp read one
+        // whole 128-byte row of a half: no bank conflict).  Otherwise raw[c]
+        // = row t, columns 8c .. 8c+7.
         Raw8<uint16_t> raw[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-            raw[c].a = lds128_addr(row_addr + (c >> 3) * kQwHalfBytes +
-                                   (((static_cast<uint32_t>(c) & 7u) ^ swz) << 4));
+        uint32_t w2[64];
         uint32_t m[16];
+        if constexpr (kTransposed) {
+            const uint32_t base = slot_addr + (cp >> 5) * kQwHalfBytes + ((cp & 3u) << 2);
+            const uint32_t chunk = (cp & 31u) >> 2;
 #pragma unroll
-        for (int c = 0; c < 16; ++c)
-            m[c] = bf16x2_absmax(bf16x2_absmax(raw[c].a.x, raw[c].a.y),
-                                 bf16x2_absmax(raw[c].a.z, raw[c].a.w));
+            for (int i = 0; i < 64; ++i) {
+                const uint32_t kr = kh * 64u + static_cast<uint32_t>(i);
+                asm volatile("ld.shared.u32 %0, [%1];"
+                             : "=r"(w2[i])
+                             : "r"(base + kr * 128u + ((chunk ^ (kr & 7u)) << 4)));
+            }
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+                m[c] = bf16x2_absmax(bf16x2_absmax(w2[4 * c], w2[4 * c + 1]),
+                                     bf16x2_absmax(w2[4 * c + 2], w2[4 * c + 3]));
+        } else {
+            const uint32_t row_addr = slot_addr + t * 128;
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+                raw[c].a = lds128_addr(row_addr + (c >> 3) * kQwHalfBytes +
+                                       (((static_cast<uint32_t>(c) & 7u) ^ swz) << 4));
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+                m[c] = bf16x2_absmax(bf16x2_absmax(raw[c].a.x, raw[c].a.y),
+                                     bf16x2_absmax(raw[c].a.z, raw[c].a.w));
+        }
 #pragma unroll
         for (int w = 8; w > 0; w >>= 1)
 #pragma unroll
@@ -172,7 +191,7 @@ __global__ void __launch_bounds__(kQwThreads, 1)
             wm = bf16x2_absmax(wm, __shfl_xor_sync(0xFFFFFFFFu, wm, off));
         const int par = static_cast<int>(k & 1);
         if (lane == 0) tail->red[g][par][wg] = wm;
-        // After this barrier every row of the block is in registers and the
+        // After this barrier every thread's values are in registers and the
         // four warp maxima are visible.
         if (!qw_group_sync(&tail->gbar[g], uses, lane, abort_flag)) break;
         uint32_t bm = bf16x2_absmax(bf16x2_absmax(tail->red[g][par][0], tail->red[g][par][1]),
@@ -186,32 +205,34 @@ __global__ void __launch_bounds__(kQwThreads, 1)
         advance(c_br, c_bc);
         const float s = scale_from_amax(amax);
         const float r = __frcp_rn(s);
-        uint32_t codes[32];
-        if (corrected_path_ok(s)) {
-            const uint64_t s2 = f2_pack(s, s);
-            const uint64_t neg_r2 = f2_pack(-r, -r);
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                uint64_t n[4];
-                raw[c].to_neg_pairs(n);
-                const uint2 cc = encode8_corrected(n, s2, neg_r2);
-                codes[2 * c] = cc.x;
-                codes[2 * c + 1] = cc.y;
-            }
-        } else {
-            // Scale off the corrected quotient's proven range: IEEE division.
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                float v[8];
-                raw[c].to_float(v);
-                codes[2 * c] = encode2_exact(v[0], v[1], s) | (encode2_exact(v[2], v[3], s) << 16);
-                codes[2 * c + 1] =
-                    encode2_exact(v[4], v[5], s) | (encode2_exact(v[6], v[7], s) << 16);
-            }
-        }
         if (t == 0) p.s[br * p.s_stride_kb + bc * p.s_stride_nb] = s;
+        const bool fast = corrected_path_ok(s);
+        const uint64_t s2 = f2_pack(s, s);
+        const uint64_t neg_r2 = f2_pack(-r, -r);
 
         if constexpr (!kTransposed) {
+            uint32_t codes[32];
+            if (fast) {
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    uint64_t n[4];
+                    raw[c].to_neg_pairs(n);
+                    const uint2 cc = encode8_corrected(n, s2, neg_r2);
+                    codes[2 * c] = cc.x;
+                    codes[2 * c + 1] = cc.y;
+                }
+            } else {
+                // Scale off the corrected quotient's proven range: IEEE division.
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    float v[8];
+                    raw[c].to_float(v);
+                    codes[2 * c] =
+                        encode2_exact(v[0], v[1], s) | (encode2_exact(v[2], v[3], s) << 16);
+                    codes[2 * c + 1] =
+                        encode2_exact(v[4], v[5], s) | (encode2_exact(v[6], v[7], s) << 16);
+                }
+            }
             uint8_t* dst = p.q + (br * 128 + t) * p.ldq + bc * 128;
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
@@ -221,37 +242,47 @@ __global__ void __launch_bounds__(kQwThreads, 1)
                 stg256_cs(dst + 32 * q4, w);
             }
         } else {
-            // Codes word gi of row t (columns 4gi..4gi+3) -> U[gi][t], in the
-            // group's transpose buffer.  Every thread finished reading the
-            // previous block's U before it passed this block's first barrier.
-            const uint32_t u_base = smem_u32(tbuf_base + g * kQwTransposeBytes);
+            // Output rows n = 2cp + j (j = 0: low bf16 of each word, 1: high),
+            // codes of block rows 64 kh .. 64 kh + 63: 8 codes per 8 rows.
 #pragma unroll
-            for (int gi = 0; gi < 32; ++gi)
-                asm volatile("st.shared.u32 [%0], %1;" ::"r"(qw_u_addr(u_base, gi, t)),
-                             "r"(codes[gi])
-                             : "memory");
-            if (!qw_group_sync(&tail->gbar[g], uses, lane, abort_flag)) break;
-            // Output row n = t: byte (n % 4) of U[n / 4][k] for k = 0..127.
-            const uint32_t gi = static_cast<uint32_t>(t) >> 2;
-            const uint32_t sel = static_cast<uint32_t>(t) & 3u;
-            // byte_perm selectors: byte `sel` of each of two words into the
-            // low two bytes, then two such halves into one word.
-            const uint32_t pick = sel | ((sel + 4u) << 4);
-            uint32_t out[32];
+            for (int j = 0; j < 2; ++j) {
+                uint32_t codes[16];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const uint4 w = lds128_addr(qw_u_addr(u_base, gi, 4u * j));
-                const uint32_t lo = __byte_perm(w.x, w.y, pick);
-                const uint32_t hi = __byte_perm(w.z, w.w, pick);
-                out[j] = __byte_perm(lo, hi, 0x5410);
-            }
-            uint8_t* dst = p.q + (bc * 128 + t) * p.ldq + br * 128;
+                for (int c = 0; c < 8; ++c) {
+                    if (fast) {
+                        uint64_t n[4];
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                const uint32_t w[8] = {out[8 * q4], out[8 * q4 + 1], out[8 * q4 + 2],
-                                       out[8 * q4 + 3], out[8 * q4 + 4], out[8 * q4 + 5],
-                                       out[8 * q4 + 6], out[8 * q4 + 7]};
-                stg256_cs(dst + 32 * q4, w);
+                        for (int q = 0; q < 4; ++q) {
+                            const uint32_t a = w2[8 * c + 2 * q], b = w2[8 * c + 2 * q + 1];
+                            const uint32_t xa = j == 0 ? a << 16 : a & 0xFFFF0000u;
+                            const uint32_t xb = j == 0 ? b << 16 : b & 0xFFFF0000u;
+                            n[q] = f2_pack(__uint_as_float(xa ^ 0x80000000u),
+                                           __uint_as_float(xb ^ 0x80000000u));
+                        }
+                        const uint2 cc = encode8_corrected(n, s2, neg_r2);
+                        codes[2 * c] = cc.x;
+                        codes[2 * c + 1] = cc.y;
+                    } else {
+                        float v[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const uint32_t a = w2[8 * c + e];
+                            v[e] = __uint_as_float(j == 0 ? a << 16 : a & 0xFFFF0000u);
+                        }
+                        codes[2 * c] =
+                            encode2_exact(v[0], v[1], s) | (encode2_exact(v[2], v[3], s) << 16);
+                        codes[2 * c + 1] =
+                            encode2_exact(v[4], v[5], s) | (encode2_exact(v[6], v[7], s) << 16);
+                    }
+                }
+                uint8_t* dst = p.q + (bc * 128 + 2 * cp + j) * p.ldq + br * 128 + kh * 64;
+#pragma unroll
+                for (int q2 = 0; q2 < 2; ++q2) {
+                    const uint32_t w[8] = {codes[8 * q2], codes[8 * q2 + 1], codes[8 * q2 + 2],
+                                           codes[8 * q2 + 3], codes[8 * q2 + 4], codes[8 * q2 + 5],
+                                           codes[8 * q2 + 6], codes[8 * q2 + 7]};
+                    stg256_cs(dst + 32 * q2, w);
+                }
             }
         }
     }
