@@ -91,11 +91,12 @@ fp8_status_t current_device(int* dev_out, int* sms_out) {
                 const void* qa_kernels[] = {
                     reinterpret_cast<const void*>(&quant_act_rows_kernel<kRowsPlain>),
                     reinterpret_cast<const void*>(&quant_act_rows_kernel<kRowsScatter>),
-                    reinterpret_cast<const void*>(&quant_weight_rows_kernel<false>),
-                    reinterpret_cast<const void*>(&quant_weight_rows_kernel<true>)};
+                    reinterpret_cast<const void*>(&quant_weight_rows_kernel<kQwBlockRows>),
+                    reinterpret_cast<const void*>(&quant_weight_rows_kernel<kQwBlockCols>),
+                    reinterpret_cast<const void*>(&quant_weight_rows_kernel<kQwColTiles>)};
                 const size_t qa_bytes[] = {kQaSmemBytes, kQaSmemBytes, kQwSmemBytes,
-                                           kQwSmemBytes};
-                for (int i = 0; i < 4; ++i) {
+                                           kQwSmemBytes, kQwSmemBytes};
+                for (int i = 0; i < 5; ++i) {
                     if (cudaFuncSetAttribute(qa_kernels[i],
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(qa_bytes[i])) != cudaSuccess) {
@@ -282,8 +283,10 @@ bool make_act_rows_map(CUtensorMap* map, const void* base, uint64_t rows, uint64
 // 128x128 quantization of a bf16 weight [K, N], one block row per thread
 // (quant_weight_rows_kernel): boxes of 128 rows x 64 columns, 128-byte
 // swizzle; one persistent CTA of kQwGroups groups per SM.
+// mode kQwColTiles: 128x1 tiles of x [K rows, N columns] (the tokens are the
+// rows), codes transposed, s[column * sb_stride_nb + band * sb_stride_kb].
 fp8_status_t launch_quant_weight_rows(const void* w, int64_t K, int64_t N, int64_t ldw,
-                                      uint8_t* q, int transpose_out, int64_t ldq, float* sb,
+                                      uint8_t* q, int mode, int64_t ldq, float* sb,
                                       int64_t sb_stride_kb, int64_t sb_stride_nb, int sms,
                                       cudaStream_t stream) {
     PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
@@ -305,10 +308,12 @@ fp8_status_t launch_quant_weight_rows(const void* w, int64_t K, int64_t N, int64
     p.s = sb; p.s_stride_kb = sb_stride_kb; p.s_stride_nb = sb_stride_nb;
     const int64_t ctas = (p.nblocks + kQwGroups - 1) / kQwGroups;
     const unsigned grid = static_cast<unsigned>(ctas < sms ? ctas : sms);
-    if (transpose_out)
-        quant_weight_rows_kernel<true><<<grid, kQwThreads, kQwSmemBytes, stream>>>(map, p);
+    if (mode == kQwColTiles)
+        quant_weight_rows_kernel<kQwColTiles><<<grid, kQwThreads, kQwSmemBytes, stream>>>(map, p);
+    else if (mode == kQwBlockCols)
+        quant_weight_rows_kernel<kQwBlockCols><<<grid, kQwThreads, kQwSmemBytes, stream>>>(map, p);
     else
-        quant_weight_rows_kernel<false><<<grid, kQwThreads, kQwSmemBytes, stream>>>(map, p);
+        quant_weight_rows_kernel<kQwBlockRows><<<grid, kQwThreads, kQwSmemBytes, stream>>>(map, p);
     return launch_status();
 }
 
@@ -616,8 +621,8 @@ fp8_status_t fp8_quantize_weight_128x128(const void* w, fp8_in_t w_type, int64_t
     // bf16 weights whose codes can leave as 32-byte stores: one block row per
     // thread.
     if (w_type == FP8_IN_BF16 && aligned32(q) && ldq % 32 == 0)
-        return launch_quant_weight_rows(w, K, N, ldw, q, transpose_out, ldq, sb, sb_stride_kb,
-                                        sb_stride_nb, sms, stream);
+        return launch_quant_weight_rows(w, K, N, ldw, q, transpose_out ? kQwBlockCols : kQwBlockRows,
+                                        ldq, sb, sb_stride_kb, sb_stride_nb, sms, stream);
     QsParams p{};
     p.rows = K; p.cols = N;
     p.nbr = K / 128; p.nbc = N / 128;
@@ -708,6 +713,10 @@ fp8_status_t fp8_quantize_act_128x1(const void* x, fp8_in_t x_type, int64_t M, i
     int dev, sms;
     fp8_status_t s = current_device(&dev, &sms);
     if (s != FP8_OK) return s;
+    // Codes that can leave as 32-byte stores: column pairs per thread.
+    if (aligned32(qt) && ldq % 32 == 0)
+        return launch_quant_weight_rows(x, M, K, ldx, qt, kQwColTiles, ldq, st, st_stride_mb,
+                                        st_stride_k, sms, stream);
     QsParams p{};
     p.rows = M; p.cols = K;
     p.nbr = M / 128; p.nbc = K / 128;

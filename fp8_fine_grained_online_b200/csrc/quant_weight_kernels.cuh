@@ -47,10 +47,16 @@ constexpr int kQwHalfBytes = 128 * 128;           // 128 rows x 64 bf16
 constexpr int kQwBlockBytes = 2 * kQwHalfBytes;   // 32 KB: a 128x128 bf16 block
 constexpr int kQwThreads = kQwGroups * 128;
 
+// Modes: 128x128 blocks with [K, N] or transposed [N, K] codes; or 128x1
+// tiles (128 rows of one column: the weight gradient's 1x128 tiles along
+// the tokens), codes transposed, one scale per column of each 128-row band.
+enum QwMode { kQwBlockRows = 0, kQwBlockCols = 1, kQwColTiles = 2 };
+
 struct QwSmemTail {
     uint64_t full[kQwGroups][kQwSlots];   // slot filled (TMA bytes)
     uint64_t gbar[kQwGroups];             // group barrier: 4 warp arrivals
     uint32_t red[kQwGroups][2][4];        // per warp packed |max|, by block parity
+    uint32_t colred[kQwGroups][2][2][64]; // 128x1: per column pair packed |max|, [parity][kh][cp]
     WaitCtl wait;
 };
 
@@ -64,6 +70,8 @@ struct QwParams {
     uint8_t* q;
     int64_t ldq;
     float* s;
+    // blocks: s[kb * s_stride_kb + nb * s_stride_nb]; 128x1 tiles:
+    // s[column * s_stride_nb + band * s_stride_kb]
     int64_t s_stride_kb, s_stride_nb;
 };
 
@@ -78,9 +86,11 @@ __device__ __forceinline__ bool qw_group_sync(uint64_t* bar, uint32_t& uses, int
     return ok;
 }
 
-template <bool kTransposed>
+template <int kMode>
 __global__ void __launch_bounds__(kQwThreads, 1)
     quant_weight_rows_kernel(const __grid_constant__ CUtensorMap tm_in, const QwParams p) {
+    constexpr bool kTransposed = kMode != kQwBlockRows;
+    constexpr bool kColScales = kMode == kQwColTiles;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     QwSmemTail* tail =
@@ -185,30 +195,51 @@ __global__ void __launch_bounds__(kQwThreads, 1)
         for (int w = 8; w > 0; w >>= 1)
 #pragma unroll
             for (int c = 0; c < w; ++c) m[c] = bf16x2_absmax(m[c], m[c + w]);
-        uint32_t wm = m[0];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-            wm = bf16x2_absmax(wm, __shfl_xor_sync(0xFFFFFFFFu, wm, off));
         const int par = static_cast<int>(k & 1);
-        if (lane == 0) tail->red[g][par][wg] = wm;
-        // After this barrier every thread's values are in registers and the
-        // four warp maxima are visible.
-        if (!qw_group_sync(&tail->gbar[g], uses, lane, abort_flag)) break;
-        uint32_t bm = bf16x2_absmax(bf16x2_absmax(tail->red[g][par][0], tail->red[g][par][1]),
-                                    bf16x2_absmax(tail->red[g][par][2], tail->red[g][par][3]));
-        bm &= 0x7FFF7FFFu;
-        const float amax = fmaxf(__uint_as_float(bm << 16), __uint_as_float(bm & 0xFFFF0000u));
+        // The block's amax (one scale), or the column pair's maxima over the
+        // band's 128 rows (two scales): this thread's half and the half of
+        // thread t ^ 64, through shared memory.
+        float sj[2], rj[2];
+        if constexpr (kColScales) {
+            tail->colred[g][par][kh][cp] = m[0];
+            if (!qw_group_sync(&tail->gbar[g], uses, lane, abort_flag)) break;
+            uint32_t cm = bf16x2_absmax(m[0], tail->colred[g][par][kh ^ 1u][cp]) & 0x7FFF7FFFu;
+            sj[0] = scale_from_amax(__uint_as_float(cm << 16));
+            sj[1] = scale_from_amax(__uint_as_float(cm & 0xFFFF0000u));
+        } else {
+            uint32_t wm = m[0];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+                wm = bf16x2_absmax(wm, __shfl_xor_sync(0xFFFFFFFFu, wm, off));
+            if (lane == 0) tail->red[g][par][wg] = wm;
+            // After this barrier every thread's values are in registers and
+            // the four warp maxima are visible.
+            if (!qw_group_sync(&tail->gbar[g], uses, lane, abort_flag)) break;
+            uint32_t bm = bf16x2_absmax(bf16x2_absmax(tail->red[g][par][0], tail->red[g][par][1]),
+                                        bf16x2_absmax(tail->red[g][par][2], tail->red[g][par][3]));
+            bm &= 0x7FFF7FFFu;
+            sj[0] = sj[1] = scale_from_amax(
+                fmaxf(__uint_as_float(bm << 16), __uint_as_float(bm & 0xFFFF0000u)));
+        }
         // The slot just read takes the block kQwSlots ahead.
         if (t == 0 && k + kQwSlots < count) issue(k + kQwSlots);
 
         const int64_t br = c_br, bc = c_bc;
         advance(c_br, c_bc);
-        const float s = scale_from_amax(amax);
-        const float r = __frcp_rn(s);
-        if (t == 0) p.s[br * p.s_stride_kb + bc * p.s_stride_nb] = s;
+        rj[0] = __frcp_rn(sj[0]);
+        rj[1] = kColScales ? __frcp_rn(sj[1]) : rj[0];
+        const float s = sj[0];
+        if constexpr (kColScales) {
+            if (kh == 0) {
+                p.s[(bc * 128 + 2 * cp) * p.s_stride_nb + br * p.s_stride_kb] = sj[0];
+                p.s[(bc * 128 + 2 * cp + 1) * p.s_stride_nb + br * p.s_stride_kb] = sj[1];
+            }
+        } else if (t == 0) {
+            p.s[br * p.s_stride_kb + bc * p.s_stride_nb] = s;
+        }
         const bool fast = corrected_path_ok(s);
         const uint64_t s2 = f2_pack(s, s);
-        const uint64_t neg_r2 = f2_pack(-r, -r);
+        const uint64_t neg_r2 = f2_pack(-rj[0], -rj[0]);
 
         if constexpr (!kTransposed) {
             uint32_t codes[32];
@@ -246,10 +277,15 @@ __global__ void __launch_bounds__(kQwThreads, 1)
             // codes of block rows 64 kh .. 64 kh + 63: 8 codes per 8 rows.
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
+                // this output row's scale: the block's, or its column's
+                const float sc = sj[j];
+                const bool fast_j = corrected_path_ok(sc);
+                const uint64_t s2j = f2_pack(sc, sc);
+                const uint64_t neg_r2j = f2_pack(-rj[j], -rj[j]);
                 uint32_t codes[16];
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    if (fast) {
+                    if (fast_j) {
                         uint64_t n[4];
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
@@ -259,7 +295,7 @@ __global__ void __launch_bounds__(kQwThreads, 1)
                             n[q] = f2_pack(__uint_as_float(xa ^ 0x80000000u),
                                            __uint_as_float(xb ^ 0x80000000u));
                         }
-                        const uint2 cc = encode8_corrected(n, s2, neg_r2);
+                        const uint2 cc = encode8_corrected(n, s2j, neg_r2j);
                         codes[2 * c] = cc.x;
                         codes[2 * c + 1] = cc.y;
                     } else {
@@ -270,9 +306,9 @@ __global__ void __launch_bounds__(kQwThreads, 1)
                             v[e] = __uint_as_float(j == 0 ? a << 16 : a & 0xFFFF0000u);
                         }
                         codes[2 * c] =
-                            encode2_exact(v[0], v[1], s) | (encode2_exact(v[2], v[3], s) << 16);
+                            encode2_exact(v[0], v[1], sc) | (encode2_exact(v[2], v[3], sc) << 16);
                         codes[2 * c + 1] =
-                            encode2_exact(v[4], v[5], s) | (encode2_exact(v[6], v[7], s) << 16);
+                            encode2_exact(v[4], v[5], sc) | (encode2_exact(v[6], v[7], sc) << 16);
                     }
                 }
                 uint8_t* dst = p.q + (bc * 128 + 2 * cp + j) * p.ldq + br * 128 + kh * 64;

@@ -59,6 +59,23 @@ def test_act_128x1_kb_major_scales_and_strides(cuda_lib, orc):
     assert np.all(untouched[:, :32] == 0xAB) and np.all(untouched[:, 32 + M:] == 0xAB)
 
 
+@pytest.mark.parametrize("M,K", [(128, 128), (384, 640), (1024, 256)])
+def test_act_128x1_column_and_stream_paths_agree(cuda_lib, orc, M, K):
+    """Codes written with 32-byte alignment take the column-pair kernel,
+    codes at a 16-byte offset the streamed box kernel: both equal the oracle
+    (codes and scales, both scale layouts) and write nothing outside qt."""
+    x = act(M, K, 3 * M + K).cuda()
+    qo, so = orc.quantize_act_128x1(to_oracle(x))
+    for offset, kb_major in ((0, False), (16, False), (0, True), (16, True)):
+        qbuf = torch.full((K, M + 16 + offset), 0xAB, dtype=torch.uint8, device="cuda")
+        qt = qbuf[:, offset:offset + M]
+        _, st = cuda_lib.fp8_quantize_act_128x1(x, qt=qt, st_kb_major=kb_major)
+        assert_codes_equal(np_u8(qt), qo)
+        assert_scales_equal((st.t() if kb_major else st).cpu().numpy(), so)
+        rest = np_u8(qbuf)
+        assert np.all(rest[:, :offset] == 0xAB) and np.all(rest[:, offset + M:] == 0xAB)
+
+
 def test_act_128x1_special_values(cuda_lib, orc):
     """Zero and -0 columns (scale 1), subnormal amax (scale off the fast
     quotient's range: IEEE division), huge amax, a column at 448, NaN
