@@ -136,19 +136,31 @@ __global__ void __launch_bounds__(kQaThreads, 1)
     }
     __syncthreads();
 
-    // Warp-major numbering across the grid (warp w of CTA b is w * grid + b),
-    // so that when the boxes do not divide evenly the surplus lands on
-    // different SMs.
+    // Plain rows: warp-major numbering across the grid (warp w of CTA b is
+    // w * grid + b, its boxes gw, gw + nw, ...), so that when the boxes do
+    // not divide evenly the surplus lands on different SMs.  Scatter: each
+    // warp takes a contiguous run of boxes (the grid's share split evenly,
+    // tiles of one row band in order), so that a band's destination rows
+    // are read once per warp and prefetched a whole band ahead.
     const int64_t gw = static_cast<int64_t>(warp) * gridDim.x + blockIdx.x;
     const int64_t nw = static_cast<int64_t>(kQaWarps) * gridDim.x;
-    const int64_t count = p.nboxes > gw ? (p.nboxes - 1 - gw) / nw + 1 : 0;
+    int64_t first, count, step_mb, step_kb;
+    if constexpr (kScatter) {
+        first = p.nboxes * gw / nw;
+        count = p.nboxes * (gw + 1) / nw - first;
+        step_mb = p.nkb == 1 ? 1 : 0;
+        step_kb = p.nkb == 1 ? 0 : 1;
+    } else {
+        first = gw;
+        count = p.nboxes > gw ? (p.nboxes - 1 - gw) / nw + 1 : 0;
+        step_mb = nw / p.nkb;
+        step_kb = nw - step_mb * p.nkb;
+    }
     uint8_t* ring = smem + warp * kQaSlots * kSlotBytes;
     uint64_t* full = tail->full[warp];
 
-    // Box b = gw + k nw is (row band b / nkb, tile b % nkb); both cursors
-    // (issue, consume) advance by nw without dividing.
-    const int64_t step_mb = nw / p.nkb;
-    const int64_t step_kb = nw - step_mb * p.nkb;
+    // Box b is (row band b / nkb, tile b % nkb); both cursors (issue,
+    // consume) advance by the warp's stride without dividing.
     auto advance = [&](int64_t& mb, int64_t& kb) {
         mb += step_mb;
         kb += step_kb;
@@ -157,8 +169,8 @@ __global__ void __launch_bounds__(kQaThreads, 1)
             ++mb;
         }
     };
-    int64_t i_mb = gw / p.nkb, i_kb = gw - (gw / p.nkb) * p.nkb;   // next box to issue
-    int64_t c_mb = i_mb, c_kb = i_kb;                               // next box to consume
+    int64_t i_mb = first / p.nkb, i_kb = first - (first / p.nkb) * p.nkb;   // next box to issue
+    int64_t c_mb = i_mb, c_kb = i_kb;                                       // next box to consume
 
     auto issue = [&](int64_t k) {   // lane 0: box k of this warp into slot k % kQaSlots
         const int slot = static_cast<int>(k % kQaSlots);
@@ -173,11 +185,12 @@ __global__ void __launch_bounds__(kQaThreads, 1)
     if (lane == 0)
         for (int64_t k = 0; k < kQaSlots && k < count; ++k) issue(k);
 
-    // Scatter form: the first kDestBatch destinations of this lane's token,
-    // for the box being processed (dst_cur) and, fetched one box ahead so
-    // that the loads' latency hides behind a whole box, the next (dst_next).
+    // Scatter form: the first kDestBatch destinations of each of the 32
+    // tokens of the band being processed (dst_cur, band dst_band) and of the
+    // band after it (dst_next), loaded when the warp enters a band.
     constexpr int kDestBatch = 8;
     int32_t dst_cur[kDestBatch], dst_next[kDestBatch];
+    int64_t dst_band = -1;
     auto load_dest = [&](int64_t mb, int32_t (&d)[kDestBatch]) {
         const int64_t row = mb * kQaRows + lane;
 #pragma unroll
@@ -185,7 +198,11 @@ __global__ void __launch_bounds__(kQaThreads, 1)
             d[j] = (row < p.rows && j < p.topk) ? __ldg(p.dest + row * p.topk + j) : -1;
     };
     if constexpr (kScatter) {
-        if (count > 0) load_dest(c_mb, dst_cur);
+        if (count > 0) {
+            load_dest(c_mb, dst_cur);
+            load_dest(c_mb + 1, dst_next);
+            dst_band = c_mb;
+        }
     }
 
     const uint32_t swz = static_cast<uint32_t>(lane & 7);
@@ -217,10 +234,8 @@ __global__ void __launch_bounds__(kQaThreads, 1)
 
         const int64_t kb = c_kb;
         const int64_t row = c_mb * kQaRows + lane;
+        const int64_t mb = c_mb;
         advance(c_mb, c_kb);
-        if constexpr (kScatter) {
-            if (k + 1 < count) load_dest(c_mb, dst_next);   // c_mb is now the next box's band
-        }
         const float s = scale_from_amax(amax);
         const float r = __frcp_rn(s);
         uint32_t codes[32];
@@ -247,6 +262,16 @@ __global__ void __launch_bounds__(kQaThreads, 1)
             }
         }
         if constexpr (kScatter) {
+            if (mb != dst_band) {   // runs advance one tile at a time: the next band
+                if (mb == dst_band + 1) {
+#pragma unroll
+                    for (int j = 0; j < kDestBatch; ++j) dst_cur[j] = dst_next[j];
+                } else {
+                    load_dest(mb, dst_cur);
+                }
+                dst_band = mb;
+                load_dest(mb + 1, dst_next);
+            }
             for (int64_t j0 = 0; j0 < p.topk; j0 += kDestBatch) {
                 int32_t dst_rows[kDestBatch];
 #pragma unroll
@@ -266,8 +291,6 @@ __global__ void __launch_bounds__(kQaThreads, 1)
                     store_row_tile(p, d, kb, codes, s);
                 }
             }
-#pragma unroll
-            for (int j = 0; j < kDestBatch; ++j) dst_cur[j] = dst_next[j];
         } else if (row < p.rows) {
             store_row_tile(p, row, kb, codes, s);
         }
