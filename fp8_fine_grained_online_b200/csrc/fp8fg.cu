@@ -203,11 +203,11 @@ inline fp8_status_t launch_status() {
     return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
-// Grouped GEMM: the CTA-pair kernel (256-row tiles) for contractions of at
-// least this many K, else the one-CTA kernel (128-row tiles).  With MoE-sized
-// groups (~256 rows) the pair's taller tiles waste more rows, which long
-// contractions amortise better (measured: K 7168 faster on the pair, K 2048
-// faster on one CTA).
+// Grouped GEMM: for contractions of at least this many K, the CTA-pair
+// kernel (256-row tiles) takes each group's whole 256-row blocks and a
+// remainder of more than 128 rows, and the one-CTA kernel a remainder of
+// 1-128 rows; shorter contractions run on the one-CTA kernel alone
+// (128-row tiles).
 constexpr int64_t kGroupedPairMinK = 4096;
 
 // L2 bytes one raster band of the dense GEMM may hold (of the B200's 126 MB;
@@ -768,8 +768,10 @@ fp8_status_t fp8_grouped_gemm(const uint8_t* a, int64_t lda, const float* sa,
     if (st != FP8_OK) return st;
     const int64_t num_nt = (N + kBN - 1) / kBN;
     const bool use_pair = K >= kGroupedPairMinK;
-    const int64_t tile_m = use_pair ? kPairBM : kBM;
-    const int64_t max_mt = total_M / tile_m + G;  // sum over groups of ceil(rows_g / tile_m)
+    // Pair tiles: sum over groups of at most ceil(rows_g / 256); the one-CTA
+    // launch: ceil(rows_g / 128) alone, or at most one tile per group after
+    // the pair launch.
+    const int64_t max_mt = use_pair ? total_M / kPairBM + G : total_M / kBM + G;
     if (total_M > INT32_MAX || max_mt * num_nt > INT32_MAX ||
         static_cast<int64_t>(G) * N > INT32_MAX)
         return FP8_ERR_SHAPE;
@@ -779,10 +781,9 @@ fp8_status_t fp8_grouped_gemm(const uint8_t* a, int64_t lda, const float* sa,
 
     CUtensorMap tmA, tmB;
     const uint64_t kcols = static_cast<uint64_t>(K);
-    const uint32_t b_box = use_pair ? 128 : kBN;   // pair: each CTA loads 128 rows of B
+    const uint64_t b_rows = static_cast<uint64_t>(G) * static_cast<uint64_t>(N);
     if (!make_operand_map(&tmA, a, static_cast<uint64_t>(total_M), kcols, static_cast<uint64_t>(lda), kBM) ||
-        !make_operand_map(&tmB, b, static_cast<uint64_t>(G) * static_cast<uint64_t>(N), kcols,
-                          static_cast<uint64_t>(ldb), b_box))
+        !make_operand_map(&tmB, b, b_rows, kcols, static_cast<uint64_t>(ldb), kBN))
         return FP8_ERR_CUDA;
 
     GemmParams p{};
@@ -796,10 +797,22 @@ fp8_status_t fp8_grouped_gemm(const uint8_t* a, int64_t lda, const float* sa,
     p.band_m = 1;
     p.band_n = 0;
     p.offsets = offsets; p.G = G;
-    if (use_pair)
-        return launch_pair_gemm<true>(tmA, tmB, p, grid_for(max_mt * num_nt, g_dev[dev].max_pairs, 1),
-                                      c_type, stream);
-    const int64_t grid = grid_for(max_mt * num_nt, sms, 1);
+    p.grp_split = kGrpAll;
+    if (use_pair) {
+        // Whole 256-row blocks (and remainders over 128 rows) on CTA pairs,
+        // then each group's remainder of 1-128 rows as one 128-row tile.
+        CUtensorMap tmB_pair;   // each CTA of a pair loads 128 rows of B
+        if (!make_operand_map(&tmB_pair, b, b_rows, kcols, static_cast<uint64_t>(ldb), 128))
+            return FP8_ERR_CUDA;
+        p.grp_split = kGrpPairPart;
+        st = launch_pair_gemm<true>(tmA, tmB_pair, p,
+                                    grid_for(max_mt * num_nt, g_dev[dev].max_pairs, 1), c_type,
+                                    stream);
+        if (st != FP8_OK) return st;
+        p.grp_split = kGrpTailPart;
+    }
+    const int64_t tail_tiles = use_pair ? static_cast<int64_t>(G) * num_nt : max_mt * num_nt;
+    const int64_t grid = grid_for(tail_tiles, sms, 1);
     if (c_type == FP8_OUT_BF16)
         blockscaled_gemm_kernel<true, true>
             <<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, stream>>>(tmA, tmB, p);

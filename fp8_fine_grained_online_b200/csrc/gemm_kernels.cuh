@@ -66,6 +66,19 @@ constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kTmemCols = 512;      // 2 partial buffers x 256 FP32 columns
 constexpr int kMaxGroups = 1024;
 
+// Grouped GEMM row split.  kGrpAll: a launch covers every row of each group
+// in tiles of its own height.  The split form covers a group's rows with
+// CTA-pair tiles of kPairRows rows except a remainder of 1 to kBM rows,
+// which a second launch of the one-CTA kernel covers with one kBM-row tile,
+// so that no group pads its last tile by more than kBM - 1 rows of MMA work
+// (a 256-row tile for a 257-row group would pad it by 255):
+//   kGrpPairPart: whole kPairRows blocks, and a remainder of more than kBM rows;
+//   kGrpTailPart: a remainder of 1 to kBM rows.
+constexpr int kGrpAll = 0;
+constexpr int kGrpPairPart = 1;
+constexpr int kGrpTailPart = 2;
+constexpr int64_t kPairRows = 256;
+
 // Status codes recorded in the device error word (values of fp8_status_t).
 constexpr unsigned kDevErrShape = 2;
 constexpr unsigned kDevErrTimeout = 9;
@@ -128,6 +141,9 @@ struct GemmParams {
     float* sc;
     int64_t sc_sm, sc_snb;
     int c_v8;        // C rows may be written as 32-byte stores (c and ldc 32-byte aligned)
+    // Grouped: which rows of each group this launch covers (kGrpAll, or one
+    // part of a split between the CTA-pair and the one-CTA kernel).
+    int grp_split;
 };
 
 // One 32-byte store of 8 words (the address 32-byte aligned).
@@ -248,6 +264,16 @@ __device__ __forceinline__ void build_group_tables(const GemmParams& p, GroupTab
             }
             lo = lo < p.M ? lo : p.M;
             hi = hi < p.M ? hi : p.M;
+            if (p.grp_split != kGrpAll) {
+                const int64_t full = (hi - lo) / kPairRows;
+                const int64_t rem = (hi - lo) - full * kPairRows;
+                if (p.grp_split == kGrpPairPart) {
+                    if (rem > 0 && rem <= kBM) hi = lo + full * kPairRows;
+                } else {   // kGrpTailPart
+                    lo += full * kPairRows;
+                    if (rem > kBM) hi = lo;
+                }
+            }
             gt->grp_lo[g] = static_cast<int>(lo);
             gt->grp_hi[g] = static_cast<int>(hi);
             tiles = static_cast<int>((hi - lo + kTileM - 1) / kTileM) * p.num_nt;

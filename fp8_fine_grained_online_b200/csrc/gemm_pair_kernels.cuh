@@ -35,6 +35,7 @@
 namespace fp8fg {
 
 constexpr int kPairBM = 256;          // rows of a pair tile
+static_assert(kPairBM == kPairRows, "grouped row split assumes pair tiles of kPairRows rows");
 constexpr int kPairStages = 6;
 constexpr int kPairHalfBytes = 128 * kBK;                // 16 KB: 128 rows x 128 B
 constexpr int kPairStageBytes = 2 * kPairHalfBytes;       // A half + B half

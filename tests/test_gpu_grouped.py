@@ -36,8 +36,10 @@ def run_grouped(cuda_lib, off, qa, sa, qb, sb, out_dtype):
                                        ([0, 0, 128], 128, 128),
                                        ([200, 56, 0, 0, 311, 129, 1, 64], 384, 256),
                                        ([1000], 512, 1024),
-                                       # long contraction: the CTA-pair kernel (256-row tiles)
-                                       ([300, 0, 17, 520, 256, 1], 256, 4096)])
+                                       # long contraction: the CTA-pair kernel (256-row
+                                       # tiles), remainders of 1-128 rows on one CTA
+                                       ([300, 0, 17, 520, 256, 1], 256, 4096),
+                                       ([400, 384, 129, 250, 0, 641, 128, 512, 383], 256, 4096)])
 def test_grouped_matches_oracle(cuda_lib, orc, sizes, N, K, out_dtype):
     off, qa, sa, qb, sb = grouped_operands(orc, sizes, N, K, sum(sizes) + N)
     c = run_grouped(cuda_lib, off, qa, sa, qb, sb, out_dtype)
