@@ -785,6 +785,11 @@ class MoE(Workload):
     def work_per_step(self):
         return 2.0 * self.R * 2 * self.I * self.H + 2.0 * self.R * self.H * self.I
 
+    def launches_per_step(self):
+        # a grouped GEMM of K >= 4096 is two launches: CTA-pair tiles, then
+        # the groups' 1-128-row remainders on the one-CTA kernel
+        return len(self.kernels) + (self.H >= 4096) + (self.I >= 4096)
+
     def step(self, marks):
         f = self.fp8
         marks(0)
@@ -1001,7 +1006,7 @@ def workload_record(wl, name, world, args, elapsed_ms, per_kernel, peaks, peak_s
     roof["traffic"] = recorded_traffic(wl.dominant, name)
     return {"config": wl.config(), "value": round(value, 3), "unit": wl.unit,
             "ms_per_step": round(elapsed_ms / args.steps, 4), "steps": args.steps,
-            "warmup": args.warmup, "gpu_launches": len(wl.kernels) * args.steps,
+            "warmup": args.warmup, "gpu_launches": wl.launches_per_step() * args.steps,
             "roofline": roof, "kernels": kernels}
 
 
