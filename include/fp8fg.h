@@ -313,6 +313,10 @@ FP8FG_API fp8_status_t fp8_blockscaled_gemm_colscale(const uint8_t* a, int64_t l
  *         FP8_ERR_SHAPE in the device error word; rows at or beyond
  *         total_M are never read or written.
  *  G      1 <= G <= 1024.
+ *  Launches: for K >= 4096 two kernels on `stream` (CTA-pair tiles of 256
+ *  rows for each group's whole 256-row blocks and remainders over 128 rows,
+ *  then one-CTA tiles of 128 rows for remainders of 1-128 rows; they write
+ *  disjoint rows of c), else one.  Both read offsets on the device.
  */
 FP8FG_API fp8_status_t fp8_grouped_gemm(const uint8_t* a, int64_t lda, const float* sa,
                               int64_t sa_stride_m, int64_t sa_stride_kb, const uint8_t* b,

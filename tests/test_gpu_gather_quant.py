@@ -68,8 +68,10 @@ def test_invalid_index_reported_and_row_untouched(cuda_lib):
 
 @pytest.mark.slow
 def test_moe_dispatch_full_size_sampled(cuda_lib, orc):
-    """8192 tokens x top-8 of 256 experts: all 65536 routed rows equal the
-    unfused gather + quantize; sampled rows against the oracle."""
+    """8192 tokens x top-8 of 256 experts: all 65536 routed rows of both
+    dispatch forms (row-order gather, token-order scatter as the MoE bench
+    runs it) equal the unfused gather + quantize; sampled rows against the
+    oracle."""
     d = synth.moe_inputs("cpu", with_weights=False)
     x = synth.act_input(8192, 7168, 1.0, 1e-3, 100.0, synth.MOE.config_id, "cpu")
     rows = d["token_of"].to(torch.int32)
@@ -77,6 +79,9 @@ def test_moe_dispatch_full_size_sampled(cuda_lib, orc):
     q, sa = cuda_lib.fp8_quantize_act_1x128_gather(xc, rc)
     q2, s2 = cuda_lib.fp8_quantize_act_1x128(xc[rc.long()].contiguous())
     assert torch.equal(q, q2) and torch.equal(sa, s2)
+    dest = synth.moe_dispatch_dest(d["token_of"], 8192, 8).cuda()
+    q3, s3 = cuda_lib.fp8_quantize_act_1x128_scatter(xc, dest, 65536)
+    assert torch.equal(q3, q2) and torch.equal(s3.view(torch.int32), s2.view(torch.int32))
     pick = np.array([0, 1, 4095, 30000, 65535])
     qo, sao = orc.quantize_act_1x128(to_oracle(x[rows[pick].long()]))
     assert_codes_equal(np_u8(q[torch.from_numpy(pick).cuda()]), qo)
@@ -89,7 +94,12 @@ def _routing(T, E, topk, seed):
 
 
 @pytest.mark.parametrize("T,E,topk,K", [(1, 4, 1, 128), (33, 8, 3, 384), (300, 16, 4, 1024),
-                                        (97, 64, 11, 256), (1024, 32, 8, 7168)])
+                                        (97, 64, 11, 256), (1024, 32, 8, 7168),
+                                        # more boxes than the grid's warps: one tile per row
+                                        # band (every box a new band), and runs of several
+                                        # boxes crossing bands
+                                        (40000, 64, 2, 128), (9000, 16, 2, 640),
+                                        (20000, 8, 2, 1024)])
 def test_scatter_quant_matches_oracle_and_gather(cuda_lib, orc, T, E, topk, K):
     """Token-order dispatch: every routed row equals the oracle's quantization
     of its token, and the whole output equals the gather form's."""
