@@ -30,6 +30,7 @@ __all__ = [
     "fp8_quantize_act_1x128_scatter",
     "fp8_blockscaled_gemm_quant", "fp8_dequantize", "fp8_quantize_act_128x1",
     "fp8_blockscaled_gemm_colscale", "linear_weight_grad", "fp8_set_wait_limit",
+    "LinearForwardPipeline",
 ]
 
 _L = _lib.lib
@@ -323,3 +324,95 @@ def e2e_linear_forward(x_host, w_host, out_host=None, device="cuda", stream=None
         out_host = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
     out_host.copy_(y, non_blocking=True)
     return out_host
+
+
+class LinearForwardPipeline:
+    """End-to-end ``linear_forward`` on host tensors, pipelined across calls.
+
+    Each ``submit(x_host, w_host, out_host)`` copies x [M, K] and w [K, N]
+    (bf16, pinned host memory) to the device on a host-to-device copy
+    stream, quantizes both and runs the block-scaled GEMM on the compute
+    stream, and copies y = x @ w [M, N] (bf16) into the pinned ``out_host``
+    on a device-to-host copy stream.  ``depth`` sets of device buffers let
+    call i+1's inputs travel while call i computes and while its result
+    travels back; the two copy directions run on separate streams, so both
+    directions of the host link are used at once.  The x quantization starts
+    as soon as x has landed, while w is still on its way.
+
+    ``submit`` only enqueues work and returns the event that completes with
+    the call's device-to-host copy.  The caller keeps ``x_host`` and
+    ``w_host`` unchanged and reads ``out_host`` only after that event (or
+    ``join`` / ``synchronize``).  ``join(stream)`` makes ``stream`` wait for
+    every submitted call; ``synchronize()`` waits on the host.
+    """
+
+    def __init__(self, M, K, N, depth=2, device="cuda", stream=None):
+        if depth < 1:
+            raise ValueError("depth must be >= 1")
+        self.M, self.K, self.N = M, K, N
+        self.compute = stream if stream is not None else torch.cuda.current_stream(device)
+        self.h2d = torch.cuda.Stream(device)
+        self.d2h = torch.cuda.Stream(device)
+        self.slots = []
+        for _ in range(depth):
+            self.slots.append(dict(
+                x=torch.empty((M, K), dtype=torch.bfloat16, device=device),
+                w=torch.empty((K, N), dtype=torch.bfloat16, device=device),
+                qx=torch.empty((M, K), dtype=torch.uint8, device=device),
+                sx=torch.empty((M, K // 128), dtype=torch.float32, device=device),
+                qw=torch.empty((N, K), dtype=torch.uint8, device=device),
+                sw=torch.empty((K // 128, N // 128), dtype=torch.float32, device=device),
+                c=torch.empty((M, N), dtype=torch.bfloat16, device=device),
+                x_in=torch.cuda.Event(), w_in=torch.cuda.Event(),
+                used=torch.cuda.Event(), out=torch.cuda.Event(), busy=False))
+        self.n = 0
+
+    def submit(self, x_host, w_host, out_host):
+        if (tuple(x_host.shape) != (self.M, self.K) or tuple(w_host.shape) != (self.K, self.N)
+                or tuple(out_host.shape) != (self.M, self.N)):
+            raise ValueError("shapes differ from the pipeline's [M, K] x [K, N]")
+        if x_host.dtype != torch.bfloat16 or w_host.dtype != torch.bfloat16 or \
+                out_host.dtype != torch.bfloat16:
+            raise TypeError("x, w and out are bfloat16")
+        s = self.slots[self.n % len(self.slots)]
+        self.n += 1
+        if s["busy"]:
+            # the slot's inputs were read by its previous call's kernels
+            self.h2d.wait_event(s["used"])
+        with torch.cuda.stream(self.h2d):
+            s["x"].copy_(x_host, non_blocking=True)
+            s["x_in"].record(self.h2d)
+            s["w"].copy_(w_host, non_blocking=True)
+            s["w_in"].record(self.h2d)
+        if s["busy"]:
+            # the slot's previous result has left the device
+            self.compute.wait_event(s["out"])
+        self.compute.wait_event(s["x_in"])
+        fp8_quantize_act_1x128(s["x"], q=s["qx"], sa=s["sx"], stream=self.compute)
+        self.compute.wait_event(s["w_in"])
+        fp8_quantize_weight_128x128(s["w"], transpose_out=True, q=s["qw"], sb=s["sw"],
+                                    stream=self.compute)
+        fp8_blockscaled_gemm(s["qx"], s["sx"], s["qw"], s["sw"], c=s["c"], stream=self.compute)
+        s["used"].record(self.compute)
+        self.d2h.wait_event(s["used"])
+        with torch.cuda.stream(self.d2h):
+            out_host.copy_(s["c"], non_blocking=True)
+            s["out"].record(self.d2h)
+        s["busy"] = True
+        return s["out"]
+
+    def join(self, stream=None):
+        """Make `stream` (default: the compute stream) wait for every call."""
+        st = stream if stream is not None else self.compute
+        st.wait_stream(self.d2h)
+        st.wait_stream(self.h2d)
+
+    def synchronize(self):
+        self.h2d.synchronize()
+        self.compute.synchronize()
+        self.d2h.synchronize()
+
+    def close(self):
+        """Wait for every call and release the device buffers."""
+        self.synchronize()
+        self.slots = []
