@@ -52,6 +52,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 FP8_OVER_BF16 = 2.0     # nominal dense ratio, 4.5 / 2.25 PFLOP/s
 CSRC = os.path.join(ROOT, "fp8_fine_grained_online_b200", "csrc")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+QUEUE_FILL_CYCLES = 400_000   # ~0.2 ms of device spin ahead of a timed region
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -942,6 +943,12 @@ def time_workload(wl, args, world, device, fp8):
     time.sleep(0.3)
     clocks.begin()
     wall0 = time.perf_counter()
+    # A short device-side spin, enqueued before the start event, keeps the
+    # GPU busy while the host enqueues the first step's launches: the region
+    # then holds the steps' GPU work, not the host's first-launch latency
+    # after the synchronize above (which had inflated the first kernel of
+    # step 0, and so its per-kernel mean, by tens of microseconds).
+    torch.cuda._sleep(QUEUE_FILL_CYCLES)
     start.record(stream)
     for s in range(args.steps):
         wl.step(lambda i, s=s: ev[s][i].record(stream))
