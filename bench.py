@@ -66,11 +66,22 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def _strip_comments(src):
+    """C/C++ source without its comments and trailing blanks (string
+    literals holding comment markers do not occur in the kernel sources)."""
+    import re
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+
+
 def kernel_source_hash():
+    """Hash of the kernel sources' code (comments and blank lines ignored),
+    the key under which profiles/dram_traffic.txt records its counters."""
     h = hashlib.sha256()
     for name in sorted(os.listdir(CSRC)):
-        with open(os.path.join(CSRC, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(CSRC, name), encoding="utf-8") as f:
+            h.update(name.encode() + _strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 

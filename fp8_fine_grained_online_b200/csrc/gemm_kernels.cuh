@@ -246,8 +246,10 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // One warp builds the grouped tile table from the device offsets: group g
-// has ceil(rows_g / kTileM) m-tiles times num_nt n-tiles.  Invalid offsets
-// (negative, or decreasing) give an empty group and record FP8_ERR_SHAPE.
+// covers the rows [grp_lo, grp_hi) this launch takes (all of them, or its
+// part of the pair / one-CTA split, kGrp*) in ceil(rows / kTileM) m-tiles
+// times num_nt n-tiles.  Invalid offsets (negative, or decreasing) give an
+// empty group and record FP8_ERR_SHAPE.
 template <int kTileM>
 __device__ __forceinline__ void build_group_tables(const GemmParams& p, GroupTables* gt, int lane,
                                                    int* total_tiles) {
@@ -293,8 +295,8 @@ __device__ __forceinline__ void build_group_tables(const GemmParams& p, GroupTab
     }
 }
 
-// Tile t of the persistent schedule.  Dense tiles are kTileM rows high;
-// grouped tiles are kBM rows of one group.
+// Tile t of the persistent schedule: kTileM rows (of one group, for the
+// grouped form) by kBN columns.
 template <bool kGrouped, int kTileM = kBM>
 __device__ __forceinline__ TileCoord decode_tile(int t, const GemmParams& p,
                                                  const GroupTables* gt) {
