@@ -58,11 +58,21 @@ QUEUE_FILL_CYCLES = 400_000   # ~0.2 ms of device spin ahead of a timed region
 # ----------------------------------------------------------------------------- helpers
 
 def load_peaks():
+    """The measured HBM copy and bf16 GEMM peaks when MEASURED_PEAKS.json is
+    present and holds them as numbers, else the fallback figures."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
-        with open(path) as f:
-            d = json.load(f)
-        return d, "measured"
+        try:
+            with open(path) as f:
+                d = json.load(f)
+            if all(isinstance(d.get(k), (int, float)) and d[k] > 0
+                   for k in ("hbm_gbs", "bf16_tflops")):
+                out = dict(FALLBACK_PEAKS)
+                out.update({k: float(v) for k, v in d.items()
+                            if k in FALLBACK_PEAKS and isinstance(v, (int, float)) and v > 0})
+                return out, "measured"
+        except (OSError, ValueError, AttributeError):
+            pass
     return dict(FALLBACK_PEAKS), "fallback"
 
 
