@@ -824,6 +824,33 @@ class MoE(Workload):
     def work_per_step(self):
         return 2.0 * self.R * 2 * self.I * self.H + 2.0 * self.R * self.H * self.I
 
+    def quant_error(self, rows=64, blocks=16, experts=4):
+        """Both grouped GEMMs of the last step on a sample (experts spread over
+        the range, rows spread within each expert, 128-column blocks spread
+        over N) against the fp64 products of the unquantized bf16 inputs and
+        that expert's bf16 weights."""
+        dev = self.cgu.device
+        off = self.off.cpu().tolist()
+        out = {}
+        for which, a, c, N in (("gate_up", None, self.cgu, 2 * self.I),
+                                  ("down", self.h, self.cdn, self.H)):
+            got, exact = [], []
+            nb = sample_index(N // 128, blocks, dev)
+            cols = (nb[:, None] * 128 + torch.arange(128, device=dev)).reshape(-1)
+            for e in sample_index(self.E, experts, "cpu").tolist():
+                lo, hi = off[e], off[e + 1]
+                if hi <= lo:
+                    continue
+                r = lo + sample_index(hi - lo, rows, dev)
+                w = synth.moe_expert_weight(e, which, dev, self.H, self.I)[:, cols].double()
+                src = self.x[self.rows[r].long()] if a is None else a[r]
+                exact.append(src.double() @ w)
+                got.append(c[r][:, cols].double())
+            out[which] = error_vs_exact(torch.cat(got), torch.cat(exact),
+                                        "%d experts x up to %d rows x %d 128-column blocks"
+                                        % (experts, rows, len(nb)))
+        return out
+
     def launches_per_step(self):
         # a grouped GEMM of K >= 4096 is two launches: CTA-pair tiles, then
         # the groups' 1-128-row remainders on the one-CTA kernel
