@@ -439,6 +439,7 @@ fp8_status_t dense_gemm(const uint8_t* a, int64_t lda, const float* sa, int64_t 
     GemmParams p = out;
     p.c_v8 = (p.c != nullptr && aligned32(p.c) &&
               (p.ldc * elem_size_out(c_type)) % 32 == 0) ? 1 : 0;
+    p.qc_v8 = (p.qc != nullptr && aligned32(p.qc) && p.ldqc % 32 == 0) ? 1 : 0;
     p.sa = sa; p.sa_sm = sa_stride_m; p.sa_skb = sa_stride_kb;
     p.sb = sb; p.sb_sg = 0; p.sb_skb = sb_stride_kb; p.sb_snb = sb_stride_nb;
     p.M = M; p.N = N;

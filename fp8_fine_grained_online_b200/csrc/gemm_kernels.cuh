@@ -141,6 +141,7 @@ struct GemmParams {
     float* sc;
     int64_t sc_sm, sc_snb;
     int c_v8;        // C rows may be written as 32-byte stores (c and ldc 32-byte aligned)
+    int qc_v8;       // code rows may be written as 32-byte stores (qc and ldqc 32-byte aligned)
     // Grouped: which rows of each group this launch covers (kGrpAll, or one
     // part of a split between the CTA-pair and the one-CTA kernel).
     int grp_split;
@@ -401,17 +402,25 @@ __device__ __forceinline__ void store_row_quantized(const GemmParams& p, const f
     for (int j = 1; j < 64; ++j) m = bf16x2_max(m, hb[j] & 0x7FFF7FFFu);
     const float amax = fmaxf(__uint_as_float(m << 16), __uint_as_float(m & 0xFFFF0000u));
     if (p.c != nullptr) {
-        uint4* out = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.c) + row * p.ldc + col0);
+        __nv_bfloat16* crow = reinterpret_cast<__nv_bfloat16*>(p.c) + row * p.ldc + col0;
+        if (p.c_v8) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-            out[j] = make_uint4(hb[4 * j], hb[4 * j + 1], hb[4 * j + 2], hb[4 * j + 3]);
+            for (int j = 0; j < 8; ++j) stg256(crow + 16 * j, hb + 8 * j);
+        } else {
+            uint4* out = reinterpret_cast<uint4*>(crow);
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                out[j] = make_uint4(hb[4 * j], hb[4 * j + 1], hb[4 * j + 2], hb[4 * j + 3]);
+        }
     }
     const float s = scale_from_amax(amax);
     const float r = __frcp_rn(s);
     const uint64_t s2 = f2_pack(s, s);
     const uint64_t neg_r2 = f2_pack(-r, -r);
     const bool fast = corrected_path_ok(s);
-    uint4* qrow = reinterpret_cast<uint4*>(p.qc + row * p.ldqc + col0);
+    uint8_t* qbase = p.qc + row * p.ldqc + col0;
+    uint4* qrow = reinterpret_cast<uint4*>(qbase);
+    uint32_t pending[4];   // the previous 16 codes, when rows take 32-byte stores
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         uint2 codes[2];
@@ -431,7 +440,20 @@ __device__ __forceinline__ void store_row_quantized(const GemmParams& p, const f
                 codes[h].y = encode2_exact(v[4], v[5], s) | (encode2_exact(v[6], v[7], s) << 16);
             }
         }
-        qrow[j] = make_uint4(codes[0].x, codes[0].y, codes[1].x, codes[1].y);
+        if (p.qc_v8) {
+            if (j & 1) {
+                const uint32_t w[8] = {pending[0], pending[1], pending[2], pending[3],
+                                       codes[0].x, codes[0].y, codes[1].x, codes[1].y};
+                stg256(qbase + 16 * (j - 1), w);
+            } else {
+                pending[0] = codes[0].x;
+                pending[1] = codes[0].y;
+                pending[2] = codes[1].x;
+                pending[3] = codes[1].y;
+            }
+        } else {
+            qrow[j] = make_uint4(codes[0].x, codes[0].y, codes[1].x, codes[1].y);
+        }
     }
     p.sc[row * p.sc_sm + (col0 / 128) * p.sc_snb] = s;
 }
