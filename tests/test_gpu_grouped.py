@@ -113,3 +113,36 @@ def test_moe_full_size_sampled(cuda_lib, orc):
                 assert_gemm_within_bound(got, C_ref, T, torch.bfloat16)
         del qb, c
     assert cuda_lib.fp8_get_device_error() == 0
+
+
+def test_max_groups_two_launch_path(cuda_lib):
+    """G = 1024 (the maximum) with random 0-300-row groups at K = 4096: the
+    CTA-pair and remainder launches both build 1024-group tile tables.  A
+    spread of groups (empty, small, over 256 rows) equals the dense GEMM of
+    the same rows with that group's weights, bit for bit."""
+    G, N, K = 1024, 256, 4096
+    rng = np.random.default_rng(11)
+    sizes = rng.integers(0, 301, G)
+    sizes[[3, 500, 1023]] = 0
+    total = int(sizes.sum())
+    off = torch.tensor(np.concatenate([[0], np.cumsum(sizes)]), dtype=torch.int32, device="cuda")
+    a = synth.normal((total, K), 1.0, 12, "cuda")
+    qa, sa = cuda_lib.fp8_quantize_act_1x128(a)
+    qb = torch.empty((G, N, K), dtype=torch.uint8, device="cuda")
+    sb = torch.empty((G, K // 128, N // 128), dtype=torch.float32, device="cuda")
+    w = synth.normal((K, G * N), 0.02, 13, "cuda")
+    for g in range(G):
+        cuda_lib.fp8_quantize_weight_128x128(w[:, g * N:(g + 1) * N], transpose_out=True,
+                                             q=qb[g], sb=sb[g])
+    c = cuda_lib.fp8_grouped_gemm(qa, sa, qb, sb, off)
+    offs = off.tolist()
+    checked = 0
+    for g in list(range(0, G, 37)) + [3, 500, 1022, 1023]:
+        lo, hi = offs[g], offs[g + 1]
+        if hi == lo:
+            continue
+        ref = cuda_lib.fp8_blockscaled_gemm(qa[lo:hi].contiguous(), sa[lo:hi].contiguous(), qb[g], sb[g])
+        assert torch.equal(c[lo:hi].view(torch.int16), ref.view(torch.int16)), g
+        checked += 1
+    assert checked > 20
+    assert cuda_lib.fp8_get_device_error() == 0
