@@ -384,6 +384,11 @@ class LinearForwardPipeline:
             s["x_in"].record(self.h2d)
             s["w"].copy_(w_host, non_blocking=True)
             s["w_in"].record(self.h2d)
+        # the caching allocator must not hand these buffers out again while
+        # the copy streams still use them (e.g. if the pipeline is dropped
+        # without close())
+        s["x"].record_stream(self.h2d)
+        s["w"].record_stream(self.h2d)
         if s["busy"]:
             # the slot's previous result has left the device
             self.compute.wait_event(s["out"])
@@ -398,6 +403,7 @@ class LinearForwardPipeline:
         with torch.cuda.stream(self.d2h):
             out_host.copy_(s["c"], non_blocking=True)
             s["out"].record(self.d2h)
+        s["c"].record_stream(self.d2h)
         s["busy"] = True
         return s["out"]
 
